@@ -1,0 +1,150 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module only draws random numbers and packs them; it contains none of
+the attention arithmetic, so both the CUDA path and the CPU oracle can be fed
+from it without sharing any of the method.
+
+Recipe (one CPU ``torch.Generator`` per workload, seeded with ``seed``):
+  1. varlen lengths: integers uniform in [lo, hi] (inclusive), one per
+     sequence, packed in draw order into int32 ``cu_seqlens``;
+  2. Q, then K, then V, then dO: i.i.d. N(0, 1) drawn in fp32, rounded to
+     bf16 (round-to-nearest-even);
+  3. optionally one query row per (batch, head) scaled by 8: the row index is
+     drawn uniformly in [0, N) after dO.  Multiplying by 8 is exact in bf16.
+Dense layout is [B, N, H, d] (d contiguous); varlen layout is [total, H, d].
+
+The named workloads mirror the shapes of the five benchmark configurations:
+GPT-2-small-shaped causal attention, BERT-large-shaped padding-free varlen
+attention, a long-sequence causal sweep, and grouped-query causal attention.
+These shapes stand in for the datasets and models of the experiments the
+pages describe; only the shapes are taken.
+"""
+import math
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+
+@dataclass
+class Workload:
+    name: str
+    B: int              # batch size, or number of sequences when varlen
+    Hq: int
+    Hkv: int
+    N: int              # sequence length, or the maximum length when varlen
+    d: int
+    causal: bool
+    scale: float
+    varlen: Optional[tuple] = None   # (lo, hi) inclusive length range
+    x8_row: bool = False             # scale one query row per head by 8
+    seed: int = 0
+    note: str = ""
+
+    def describe(self):
+        out = dict(B=self.B, Hq=self.Hq, Hkv=self.Hkv, N=self.N, d=self.d,
+                   causal=self.causal, scale=self.scale)
+        if self.varlen:
+            out["varlen_lengths"] = list(self.varlen)
+        if self.x8_row:
+            out["x8_query_row_per_head"] = True
+        return out
+
+
+def _w(name, B, H, N, d, causal, Hkv=None, **kw):
+    return Workload(name=name, B=B, Hq=H, Hkv=H if Hkv is None else Hkv, N=N, d=d,
+                    causal=causal, scale=1.0 / math.sqrt(d), **kw)
+
+
+WORKLOADS = {
+    "single_head_n128_d64": _w("single_head_n128_d64", 1, 1, 128, 64, False),
+    "gpt2_small_causal_b8_h12_n1024_d64": _w("gpt2_small_causal_b8_h12_n1024_d64",
+                                             8, 12, 1024, 64, True),
+    "bert_large_varlen_32x128to512_h16_d64": _w("bert_large_varlen_32x128to512_h16_d64",
+                                                32, 16, 512, 64, False, varlen=(128, 512)),
+    "gqa_causal_b2_hq32_hkv8_n4096_d128": _w("gqa_causal_b2_hq32_hkv8_n4096_d128",
+                                             2, 32, 4096, 128, True, Hkv=8),
+}
+for _d in (64, 128):
+    for _n in (4096, 16384, 65536):
+        _name = "long_causal_b1_h16_n%d_d%d_x8row" % (_n, _d)
+        WORKLOADS[_name] = _w(_name, 1, 16, _n, _d, True, x8_row=True)
+
+
+@dataclass
+class Inputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    dout: torch.Tensor
+    cu_seqlens: Optional[torch.Tensor]
+    workload: Workload
+    x8_rows: Optional[torch.Tensor] = None   # [B, Hq] row index scaled by 8
+    lengths: Optional[list] = field(default=None)
+
+    @property
+    def total(self):
+        return self.q.shape[0] if self.cu_seqlens is not None else self.q.shape[0] * self.q.shape[1]
+
+
+def generate(w: Workload, with_dout: bool = True) -> Inputs:
+    """Draw the inputs of workload ``w`` on the CPU (bf16 tensors)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    cu = None
+    lengths = None
+    if w.varlen:
+        lo, hi = w.varlen
+        lens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64)
+        lengths = [int(x) for x in lens]
+        cu = torch.zeros(w.B + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+        total = int(cu[-1])
+        qshape, kshape = (total, w.Hq, w.d), (total, w.Hkv, w.d)
+    else:
+        qshape, kshape = (w.B, w.N, w.Hq, w.d), (w.B, w.N, w.Hkv, w.d)
+    q = torch.randn(qshape, generator=g, dtype=torch.float32)
+    k = torch.randn(kshape, generator=g, dtype=torch.float32)
+    v = torch.randn(kshape, generator=g, dtype=torch.float32)
+    dout = torch.randn(qshape, generator=g, dtype=torch.float32) if with_dout else None
+    x8 = None
+    if w.x8_row:
+        if w.varlen:
+            raise ValueError("x8 rows are defined for dense workloads only")
+        x8 = torch.randint(0, w.N, (w.B, w.Hq), generator=g, dtype=torch.int64)
+        for b in range(w.B):
+            for h in range(w.Hq):
+                q[b, int(x8[b, h]), h, :] *= 8.0
+    bf = torch.bfloat16
+    return Inputs(q=q.to(bf), k=k.to(bf), v=v.to(bf),
+                  dout=None if dout is None else dout.to(bf),
+                  cu_seqlens=cu, workload=w, x8_rows=x8, lengths=lengths)
+
+
+def custom(name, B, Hq, Hkv, N, d, causal, scale=None, varlen=None, x8_row=False, seed=0):
+    """An ad-hoc workload (tests use this for edge shapes)."""
+    return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, causal=causal,
+                    scale=(1.0 / math.sqrt(d)) if scale is None else scale,
+                    varlen=varlen, x8_row=x8_row, seed=seed)
+
+
+def from_lengths(name, lengths, Hq, Hkv, d, causal, seed=0):
+    """Varlen inputs with explicitly given sequence lengths (edge cases such
+    as 0, 1 and 129); the values follow the same Q, K, V, dO draw order."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    lens = torch.tensor(lengths, dtype=torch.int64)
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    total = int(cu[-1])
+    q = torch.randn((total, Hq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((total, Hkv, d), generator=g, dtype=torch.float32)
+    v = torch.randn((total, Hkv, d), generator=g, dtype=torch.float32)
+    dout = torch.randn((total, Hq, d), generator=g, dtype=torch.float32)
+    w = Workload(name=name, B=len(lengths), Hq=Hq, Hkv=Hkv,
+                 N=max(lengths) if lengths else 0, d=d, causal=causal,
+                 scale=1.0 / math.sqrt(d), varlen=(min(lengths), max(lengths)) if lengths else (0, 0),
+                 seed=seed)
+    bf = torch.bfloat16
+    return Inputs(q=q.to(bf), k=k.to(bf), v=v.to(bf), dout=dout.to(bf), cu_seqlens=cu,
+                  workload=w, lengths=list(lengths))

@@ -1,0 +1,74 @@
+"""The FLOP / byte accounting reproduces the figures the pages print.
+
+Fixture: tests/golden/page_figures.json (each entry cites its page and
+section).  CPU only.
+"""
+import json
+import os
+
+import pytest
+
+from exact_io_aware_67_b200 import flops, workloads
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")))
+
+
+def _parse(s, binary):
+    num, unit = s.split()
+    if binary:
+        return float(num) * {"MB": 2 ** 20, "GB": 2 ** 30}[unit]
+    return float(num) * {"MB": 1e6, "GB": 1e9}[unit]
+
+
+@pytest.mark.parametrize("row", GOLD["standard_attention_table"]["rows"])
+def test_flop_column(row):
+    d = GOLD["standard_attention_table"]["d"]
+    f = flops.standard_attention_flops(row["N"], d)
+    # the page rounds to 2-3 significant digits
+    assert abs(f / 1e9 - row["gflops"]) <= 0.006 * row["gflops"] + 0.005
+
+
+@pytest.mark.parametrize("row", GOLD["standard_attention_table"]["rows"])
+def test_traffic_and_memory_columns(row):
+    d = GOLD["standard_attention_table"]["d"]
+    N = row["N"]
+    # traffic column: 4N^2 + 4Nd elements at one byte each (the page's own
+    # arithmetic), i.e. half of our fp16 byte count
+    t = flops.standard_attention_hbm_bytes(N, d, elem_bytes=1)
+    assert abs(t / _parse(row["traffic"], binary=False) - 1) < 0.065
+    # intermediate column: S and P of N^2 fp16 values each = 4 N^2 bytes
+    assert abs(4.0 * N * N / _parse(row["intermediate"], binary=True) - 1) < 1e-9
+
+
+def test_page1_io_example():
+    ex = GOLD["io_example"]
+    N, d = ex["N"], ex["d"]
+    assert abs(3 * N * d * 2 / 2 ** 20 - 3.0) < 1e-9
+    assert abs(N * N * 2 / 2 ** 20 - 32.0) < 1e-9
+
+
+def test_workload_flop_counts():
+    w = workloads.WORKLOADS["gqa_causal_b2_hq32_hkv8_n4096_d128"]
+    assert flops.fwd_flops(w) == 0.5 * 4 * 2 * 32 * 4096 ** 2 * 128
+    assert abs(flops.fwd_flops(w) / 1e9 - 274.9) < 0.1
+    assert flops.bwd_flops(w) == 2.5 * flops.fwd_flops(w)
+    w2 = workloads.WORKLOADS["gpt2_small_causal_b8_h12_n1024_d64"]
+    assert abs(flops.fwd_flops(w2) / 1e9 - 12.88) < 0.01
+    w4 = workloads.WORKLOADS["long_causal_b1_h16_n65536_d128_x8row"]
+    assert abs(flops.fwd_flops(w4) / 1e9 - 17592) < 1
+    wv = workloads.WORKLOADS["bert_large_varlen_32x128to512_h16_d64"]
+    lens = [128, 512]
+    assert flops.fwd_flops(wv, lens) == 4 * 16 * 64 * (128 ** 2 + 512 ** 2)
+
+
+def test_generator_is_deterministic_and_ordered():
+    w = workloads.custom("t", 1, 2, 1, 16, 8, True, x8_row=True)
+    a = workloads.generate(w)
+    b = workloads.generate(w)
+    for x, y in ((a.q, b.q), (a.k, b.k), (a.v, b.v), (a.dout, b.dout)):
+        assert (x.float() == y.float()).all()
+    assert a.x8_rows.shape == (1, 2)
+    wv = workloads.WORKLOADS["bert_large_varlen_32x128to512_h16_d64"]
+    iv = workloads.generate(wv)
+    assert len(iv.lengths) == 32 and all(128 <= L <= 512 for L in iv.lengths)
+    assert int(iv.cu_seqlens[-1]) == sum(iv.lengths) == iv.q.shape[0]
