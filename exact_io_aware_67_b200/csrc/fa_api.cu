@@ -1,0 +1,229 @@
+// fa_api.cu -- host side of libfa.so: argument validation, TMA descriptor
+// encoding, launch configuration, and the C entry points declared in
+// include/fa.h.  The library allocates no device memory and never
+// synchronises the caller's stream.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
+  if (f == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && ptr != nullptr) {
+      f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+      fn.store(f);
+    }
+  }
+  return f;
+}
+
+// Tensor map over a token-major bf16 tensor [batches][rows][heads][d]:
+// box = 64 d-elements (128 B, 128-byte swizzle) x 1 head x 128 rows.
+// Rows past `rows` read as zeros.
+bool encode_rows_map(CUtensorMap* m, const void* base, int d, int heads, long rows,
+                     int batches) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows,
+                              (cuuint64_t)batches};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2,
+                                 (cuuint64_t)rows * heads * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r =
+      enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Dims {
+  int B, Hq, Hkv, N, d, total;
+  bool varlen;
+  long rows() const { return varlen ? (long)total : (long)N; }
+  int batches() const { return varlen ? 1 : B; }
+  long tokens() const { return varlen ? (long)total : (long)B * N; }
+};
+
+// Shared validation of the size arguments.  Returns FA_OK and sets *empty
+// when there is nothing to compute.
+fa_status check_dims(const Dims& s, float scale, bool* empty) {
+  *empty = false;
+  if (s.d != 64 && s.d != 128) return FA_ERR_UNSUPPORTED;
+  if (s.B < 0 || s.Hq < 1 || s.Hkv < 1 || s.Hq % s.Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (s.N < 1 || s.N > (1 << 24)) return FA_ERR_INVALID_ARG;
+  if (s.varlen && s.total < 0) return FA_ERR_INVALID_ARG;
+  if (s.Hq > 65535) return FA_ERR_INVALID_ARG;
+  if (s.B == 0 || (s.varlen && s.total == 0)) {
+    *empty = true;
+    return FA_OK;
+  }
+  const long long qblocks = (s.N + 255) / 256;
+  if (qblocks * s.Hq * s.B > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (s.tokens() * s.Hq * (long long)s.d > (1LL << 40)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const fa::FwdParams& p, cudaStream_t stream) {
+  auto kern = fa::fwd_kernel<D, CAUSAL>;
+  const int smem = fa::FwdLayout<D>::ALLOC;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)p.num_qblocks * p.Hq * p.B;
+  kern<<<grid, fa::FWD_THREADS, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
+                 int total_tokens, cudaStream_t stream) {
+  const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
+  bool empty = false;
+  fa_status st = check_dims(s, scale, &empty);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+
+  CUtensorMap mq, mk, mv;
+  if (!encode_rows_map(&mq, q, d, Hq, s.rows(), s.batches()) ||
+      !encode_rows_map(&mk, k, d, Hkv, s.rows(), s.batches()) ||
+      !encode_rows_map(&mv, v, d, Hkv, s.rows(), s.batches()))
+    return FA_ERR_CUDA;
+
+  fa::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.total = s.varlen ? total_tokens : B * N;
+  p.num_qblocks = (N + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+
+  cudaError_t e;
+  if (d == 64)
+    e = causal ? launch_fwd<64, true>(mq, mk, mv, p, stream)
+               : launch_fwd<64, false>(mq, mk, mv, p, stream);
+  else
+    e = causal ? launch_fwd<128, true>(mq, mk, mv, p, stream)
+               : launch_fwd<128, false>(mq, mk, mv, p, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
+  if (B < 0 || Hq < 1 || N < 1 || (d != 64 && d != 128) || total_tokens < 0) return 0;
+  return fa::bwd_workspace_bytes(Hq, d, (long)total_tokens);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
+  const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
+  bool empty = false;
+  fa_status st = check_dims(s, scale, &empty);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  const size_t need = fa::bwd_workspace_bytes(Hq, d, s.tokens());
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_WORKSPACE;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (!encode_rows_map(&mq, q, d, Hq, s.rows(), s.batches()) ||
+      !encode_rows_map(&mk, k, d, Hkv, s.rows(), s.batches()) ||
+      !encode_rows_map(&mv, v, d, Hkv, s.rows(), s.batches()) ||
+      !encode_rows_map(&mdo, dO, d, Hq, s.rows(), s.batches()))
+    return FA_ERR_CUDA;
+
+  fa::BwdParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dO);
+  p.lse = lse;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.total = s.varlen ? total_tokens : B * N;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  fa::bwd_carve_workspace(p, workspace, s.tokens(), d);
+
+  const cudaError_t e = fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_device_error(void) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_error, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+fa_status fa_clear_device_error(void) {
+  const int z = 0;
+  return cudaMemcpyToSymbol(fa::g_fa_error, &z, sizeof(int)) == cudaSuccess ? FA_OK
+                                                                             : FA_ERR_CUDA;
+}
+
+void fa_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns.store(ns < 1000ull ? 1000ull : ns);
+}
+
+fa_status fa_watchdog_selftest(cudaStream_t stream) {
+  fa::watchdog_selftest_kernel<<<1, 32, 0, stream>>>(g_wait_limit_ns.load());
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+  }
+  return "FA_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

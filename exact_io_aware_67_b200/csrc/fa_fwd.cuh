@@ -1,0 +1,377 @@
+// fa_fwd.cuh -- forward attention kernel for sm_100a.
+//
+// Computes O = softmax(scale Q K^T + mask) V and LSE for one block of 256
+// query rows of one (sequence, query head) per CTA, streaming K and V tiles
+// of 128 rows through shared memory ("FlashAttention优化" 3.1: Q blocks stay
+// on chip while K/V blocks stream past; paper review 方法 item 1: no N x N
+// matrix is written back, only O).  The softmax statistics follow the online
+// recurrence of "FlashAttention优化" 3.2.1 (running max m, running sum l,
+// l <- e^(m_old - m_new) l + sum exp(x - m_new)) and the accumulated output
+// is rescaled by the same factor (paper review 方法 item 2).
+//
+// B200 design (not the pages' A100 r = c = 64 design):
+//  * Two 128-row Q tiles per CTA share every K/V tile (halves L2->SMEM
+//    traffic) and ping-pong on the tensor core: while softmax works on
+//    tile 0, the MMA warp runs tile 1's products and vice versa.
+//  * S = Q K^T and O += P V run as tcgen05.mma (M = 128) with fp32
+//    accumulators in TMEM: S_t at columns [128 t, 128 t + 128), O_t at
+//    [256 + d t, 256 + d t + d).  P (bf16) overwrites the first 64 columns of
+//    S_t and feeds the PV product straight from TMEM.
+//  * One TMA warp fills a ring of K/V stages (mbarrier full/empty pairs),
+//    one thread issues all MMAs, and each softmax warpgroup owns one Q tile:
+//    a thread owns one query row (TMEM lane), so row max and row sum are
+//    in-thread reductions.
+//  * Exponentials are exp2 with the scale folded in (x = s scale log2 e).
+//    The running max is only moved when the tile max exceeds it by more than
+//    RESCALE_LOG2 (factor 256); otherwise the stale max is kept for both O
+//    and l, which is exact because the final O / l uses the same reference.
+//    O in TMEM is then rescaled only for rows whose max moved.
+//  * Causal attention skips every K/V tile above the diagonal; only the
+//    last tile of each Q tile is masked element-wise.  Variable-length
+//    batches mask key columns past the sequence end and never store rows
+//    past it.
+#pragma once
+#include "fa_common.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int TILE = 128 * D * 2;     // bytes of one 128 x D bf16 tile
+  static constexpr int NS = (D == 128) ? 3 : 6;  // K/V ring stages
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_RING + NS * TILE;
+  // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_done[2] drain[1]
+  static constexpr int NBAR = 2 + 2 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
+};
+
+constexpr int FWD_THREADS = 320;   // warps 0-7 softmax, 8 TMA, 9 MMA
+constexpr float RESCALE_LOG2 = 8.0f;
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(FWD_THREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  constexpr int NS = L::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------------- work item
+  const int bh = p.B * p.Hq;
+  const int qb = p.num_qblocks - 1 - (int)(blockIdx.x / bh);   // heaviest blocks first
+  const int h = (int)(blockIdx.x % bh) % p.Hq;
+  const int b = (int)(blockIdx.x % bh) / p.Hq;
+  int seq_start = 0, len = p.N, bcoord = b;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - seq_start;
+    bcoord = 0;
+  }
+  const int q0 = qb * 256;
+  if (q0 >= len) return;
+  const int hk = h / p.group;
+  const int nkv_all = (len + 127) / 128;
+  int n_t[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int r0 = q0 + 128 * t;
+    n_t[t] = (r0 >= len) ? 0 : (CAUSAL ? min(nkv_all, r0 / 128 + 1) : nkv_all);
+  }
+  const int nmax = max(n_t[0], n_t[1]);
+
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* ring = smem + L::OFF_RING;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = kv_full + NS;
+  uint64_t* s_full = kv_empty + NS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 128);
+      mbar_init(o_done + i, 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_empty + s, 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
+
+  if (warp == 8) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (n_t[t] == 0) continue;
+        mbar_arrive_expect_tx(q_full + t, L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sQ + t * L::TILE + c * 16384, &tmQ, q_full + t, c * 64, h,
+                      seq_start + q0 + 128 * t, bcoord);
+      }
+      int issued = 0;
+      for (int n = 0; n < 2 * nmax; ++n) {
+        const int stage = n % NS;
+        if (!mbar_wait(kv_empty + stage, ((n / NS) & 1) ^ 1, wd, ERR_FWD_KV_EMPTY)) break;
+        const CUtensorMap* map = (n & 1) ? &tmV : &tmK;
+        mbar_arrive_expect_tx(kv_full + stage, L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(ring + stage * L::TILE + c * 16384, map, kv_full + stage, c * 64, hk,
+                      seq_start + 128 * (n >> 1), bcoord);
+        issued = n + 1;
+      }
+      if (*abort_flag) {
+        // loads still in flight must land before the CTA may exit
+        for (int n = max(0, issued - NS); n < issued; ++n)
+          mbar_wait_drain(kv_full + n % NS, (n / NS) & 1, p.wait_limit_ns);
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) mbar_wait_drain(q_full + t, 0, p.wait_limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t ring_addr = smem_u32(ring);
+      // S_t = Q_t K^T : A = Q_t (K-major), B = K tile (K-major), K-dim = d
+      auto issue_s = [&](int t, int stage) {
+        const uint32_t dt = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(dt, sdesc_sw128(q_addr + t * L::TILE + off, 16, 1024),
+                 sdesc_sw128(ring_addr + stage * L::TILE + off, 16, 1024), idesc_s, kk > 0);
+        }
+      };
+      // O_t (+)= P_t V : A = P_t from TMEM, B = V tile (N = d contiguous)
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t dt = tmem + 256 + t * D;
+        const uint32_t at = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(dt, at + kk * 8, sdesc_sw128(ring_addr + stage * L::TILE + kk * 2048, 16384, 1024),
+                 idesc_o, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = true;
+      for (int t = 0; t < 2 && ok; ++t)
+        if (n_t[t] > 0) ok = mbar_wait(q_full + t, 0, wd, ERR_FWD_Q_FULL);
+      if (ok) ok = mbar_wait(kv_full + 0, 0, wd, ERR_FWD_KV_FULL);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (n_t[t] > 0) {
+            issue_s(t, 0);
+            mma_commit(s_full + t);
+          }
+        mma_commit(kv_empty + 0);
+      }
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int nv = 2 * j + 1, sv = nv % NS;
+        const int nk = 2 * j + 2, sk = nk % NS;
+        const bool has_next = j + 1 < nmax;
+        if (!(ok = mbar_wait(kv_full + sv, (nv / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
+        tc_fence_after();
+        if (j < n_t[0]) {
+          if (!(ok = mbar_wait(p_full + 0, j & 1, wd, ERR_FWD_P_FULL))) break;
+          tc_fence_after();
+          issue_pv(0, sv, j > 0);
+          if (j == n_t[0] - 1) mma_commit(o_done + 0);
+        }
+        if (has_next) {
+          if (!(ok = mbar_wait(kv_full + sk, (nk / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
+          tc_fence_after();
+          if (j + 1 < n_t[0]) {
+            issue_s(0, sk);
+            mma_commit(s_full + 0);
+          }
+        }
+        if (j < n_t[1]) {
+          if (!(ok = mbar_wait(p_full + 1, j & 1, wd, ERR_FWD_P_FULL))) break;
+          tc_fence_after();
+          issue_pv(1, sv, j > 0);
+          if (j == n_t[1] - 1) mma_commit(o_done + 1);
+        }
+        mma_commit(kv_empty + sv);
+        if (has_next) {
+          if (j + 1 < n_t[1]) {
+            issue_s(1, sk);
+            mma_commit(s_full + 1);
+          }
+          mma_commit(kv_empty + sk);
+        }
+      }
+      // every MMA issued above completes before TMEM can be released
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ softmax
+    const int t = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;                 // row in tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const int qrow = q0 + 128 * t + r;
+    const float c2 = p.scale_log2;
+    const int n = n_t[t];
+    float m = -INFINITY;   // running max of s * scale * log2(e)
+    float l = 0.f;         // running sum of exp2(x - m)
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full + t, j & 1, wd, ERR_FWD_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(tS + 0, s + 0);
+      tmem_ld32(tS + 32, s + 32);
+      tmem_ld32(tS + 64, s + 64);
+      tmem_ld32(tS + 96, s + 96);
+      tmem_wait_ld32(s + 0);
+      tmem_wait_ld32(s + 32);
+      tmem_wait_ld32(s + 64);
+      tmem_wait_ld32(s + 96);
+      if (j == n - 1) {
+        // last tile of this Q tile: sequence end and/or causal diagonal
+        int lim = len - 128 * j;
+        if (CAUSAL) lim = min(lim, qrow + 1 - 128 * j);
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) s[c] = 0xff800000u;   // -inf
+      }
+      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_tile > m + RESCALE_LOG2) {
+        alpha = ex2(m - m_tile);   // 0 on the first tile (m = -inf)
+        resc = (j > 0);
+        m = m_tile;
+      }
+      l *= alpha;
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(s[32 * cc + 2 * i]), c2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(s[32 * cc + 2 * i + 1]), c2, neg_m));
+          l0 += p0;
+          l1 += p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + 16 * cc, pk);
+      }
+      l += l0 + l1;
+      tmem_wait_st();
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_t holds PV of all earlier tiles (S_t of this tile was issued
+        // after them), so it can be rescaled in place now.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld32(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(p_full + t);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && n > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(o_done + t, 0, wd, ERR_FWD_O_DONE));
+      if (ok) {
+        tc_fence_after();
+        const bool row_ok = qrow < len;
+        const float inv_l = 1.f / l;
+        const long tok = (p.cu_seqlens != nullptr) ? (long)seq_start + qrow
+                                                    : (long)b * p.N + qrow;
+        __nv_bfloat16* orow = p.o + (tok * p.Hq + h) * (long)D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld32(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv_l,
+                              __uint_as_float(o[2 * i + 1]) * inv_l);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+        if (row_ok) {
+          const float lse = (m + log2f(l)) * 0.69314718055994530942f;
+          const long li = (p.cu_seqlens != nullptr) ? (long)h * p.total + seq_start + qrow
+                                                    : ((long)b * p.Hq + h) * p.N + qrow;
+          p.lse[li] = lse;
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

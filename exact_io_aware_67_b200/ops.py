@@ -1,0 +1,215 @@
+"""Python binding of libfa.so -- argument marshalling only.
+
+The functions named ``fa_*`` mirror the C entry points of ``include/fa.h``
+one to one (plain integers and device pointers).  ``attention_fwd`` and
+``attention_bwd`` are conveniences that take torch CUDA tensors, allocate the
+outputs and the workspace with torch, and call the C entry points on the
+current torch stream.  Every step of the computation runs in the CUDA
+kernels of libfa.so; there is no other implementation behind this module,
+and it raises if the library cannot be loaded.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_lib = None
+
+FA_OK = 0
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
+          3: "FA_ERR_WORKSPACE", 4: "FA_ERR_CUDA"}
+
+EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
+            "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
+            "fa_status_string"]
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__("%s failed: %s" % (fn, STATUS.get(status, status)))
+        self.status = status
+
+
+def lib_path():
+    return _build.LIB
+
+
+def load(build_if_missing=True):
+    """Load libfa.so (building it first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB
+    if build_if_missing:
+        path = _build.build()
+    if not os.path.exists(path):
+        raise RuntimeError("libfa.so not found at %s; run python -m exact_io_aware_67_b200.build"
+                           % path)
+    lib = ctypes.CDLL(path)
+    vp, ip, c_int, c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp] + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
+    lib.fa_fwd.restype = c_int
+    lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t] + [c_int] * 5 + \
+        [c_float, c_int, vp, c_int, vp]
+    lib.fa_bwd.restype = c_int
+    lib.fa_bwd_workspace_size.argtypes = [c_int] * 5
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_device_error.argtypes = []
+    lib.fa_device_error.restype = c_int
+    lib.fa_clear_device_error.argtypes = []
+    lib.fa_clear_device_error.restype = c_int
+    lib.fa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.fa_set_wait_limit_ns.restype = None
+    lib.fa_watchdog_selftest.argtypes = [vp]
+    lib.fa_watchdog_selftest.restype = c_int
+    lib.fa_status_string.argtypes = [c_int]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    if os.environ.get("FA_WAIT_LIMIT_NS"):
+        lib.fa_set_wait_limit_ns(int(os.environ["FA_WAIT_LIMIT_NS"]))
+    _lib = lib
+    return lib
+
+
+# ------------------------------------------------------------ raw C entry points
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, total_tokens, stream):
+    return load().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, int(causal), cu_seqlens,
+                         total_tokens, stream)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+           scale, causal, cu_seqlens, total_tokens, stream):
+    return load().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq,
+                         Hkv, N, d, scale, int(causal), cu_seqlens, total_tokens, stream)
+
+
+def fa_bwd_workspace_size(B, Hq, N, d, total_tokens):
+    return load().fa_bwd_workspace_size(B, Hq, N, d, total_tokens)
+
+
+def fa_device_error():
+    return load().fa_device_error()
+
+
+def fa_clear_device_error():
+    return load().fa_clear_device_error()
+
+
+def fa_set_wait_limit_ns(ns):
+    load().fa_set_wait_limit_ns(int(ns))
+
+
+def fa_watchdog_selftest(stream):
+    return load().fa_watchdog_selftest(stream)
+
+
+def fa_status_string(s):
+    return load().fa_status_string(int(s)).decode()
+
+
+# ------------------------------------------------------------ torch conveniences
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _shape(q, k, cu_seqlens, max_seqlen):
+    if cu_seqlens is None:
+        B, N, Hq, d = q.shape
+        Hkv = k.shape[2]
+        total = B * N
+    else:
+        total, Hq, d = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("varlen inputs need max_seqlen (no device->host read is made)")
+        N = int(max_seqlen)
+    return B, Hq, Hkv, N, d, total
+
+
+def _check(t, name, dtype=torch.bfloat16):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
+
+
+def attention_fwd(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None,
+                  out=None, lse=None):
+    """O, LSE = fa_fwd(q, k, v).  Dense [B, N, H, d] or varlen [total, H, d]."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, nm)
+    B, Hq, Hkv, N, d, total = _shape(q, k, cu_seqlens, max_seqlen)
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N) if cu_seqlens is None else (Hq, total),
+                          dtype=torch.float32, device=q.device)
+    if cu_seqlens is not None:
+        _check(cu_seqlens, "cu_seqlens", torch.int32)
+    st = fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                float(scale), causal, _ptr(cu_seqlens), total, _stream())
+    if st != FA_OK:
+        raise FAError("fa_fwd", st)
+    return out, lse
+
+
+def workspace_for(q, k, cu_seqlens=None, max_seqlen=None):
+    """A torch-allocated workspace of fa_bwd_workspace_size() bytes."""
+    B, Hq, _, N, d, total = _shape(q, k, cu_seqlens, max_seqlen)
+    nbytes = fa_bwd_workspace_size(B, Hq, N, d, total)
+    return torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+
+
+def attention_bwd(q, k, v, out, lse, dout, scale=None, causal=False, cu_seqlens=None,
+                  max_seqlen=None, workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV = fa_bwd(...), recomputing P from the forward's LSE."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, nm)
+    _check(lse, "lse", torch.float32)
+    B, Hq, Hkv, N, d, total = _shape(q, k, cu_seqlens, max_seqlen)
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, N, d, total), dtype=torch.uint8,
+                                device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, N, d, float(scale),
+                causal, _ptr(cu_seqlens), total, _stream())
+    if st != FA_OK:
+        raise FAError("fa_bwd", st)
+    return dq, dk, dv
+
+
+class Attention(torch.autograd.Function):
+    """Autograd wrapper: forward saves Q, K, V, O and LSE (O(N) memory) and
+    the backward recomputes P in fa_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal, cu_seqlens, max_seqlen):
+        o, lse = attention_fwd(q, k, v, scale, causal, cu_seqlens, max_seqlen)
+        ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
+        ctx.scale, ctx.causal, ctx.max_seqlen = scale, causal, max_seqlen
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, cu = ctx.saved_tensors
+        dq, dk, dv = attention_bwd(q, k, v, o, lse, do.contiguous(), ctx.scale, ctx.causal,
+                                   cu, ctx.max_seqlen)
+        return dq, dk, dv, None, None, None, None
+
+
+def attention(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None):
+    return Attention.apply(q, k, v, scale if scale is not None else q.shape[-1] ** -0.5,
+                           causal, cu_seqlens, max_seqlen)

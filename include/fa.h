@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact IO-aware attention on NVIDIA B200
+ * (sm_100a).  Forward writes O and the per-row log-sum-exp; backward
+ * recomputes S and P from Q, K, V and that LSE and returns dQ, dK, dV.
+ * No N x N score or probability matrix is ever written to device memory.
+ *
+ * What is computed ("注意力机制基础", section 2.1; "FlashAttention优化",
+ * sections 3.1-3.2; "FlashAttention: Fast and Memory-Efficient Exact
+ * Attention with IO-Awareness" review, 方法 items 1-3):
+ *     S   = scale * Q K^T, with key j > query i set to -inf when causal
+ *     P   = row softmax(S),  O = P V,  LSE_i = ln(sum_j exp(S_ij))
+ * computed tile by tile with the online-softmax running max and sum.  The
+ * backward is the derivative of the same definition:
+ *     dV = P^T dO,  dP = dO V^T,  D_i = sum_k dO_ik O_ik,
+ *     dS = P o (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+ *
+ * Common argument conventions
+ *   q, o, dO, dq : bf16, dense [B][N][Hq][d] or varlen [total][Hq][d]
+ *   k, v, dk, dv : bf16, dense [B][N][Hkv][d] or varlen [total][Hkv][d]
+ *                  (d contiguous; rows of one token are Hq*d or Hkv*d apart)
+ *   lse          : fp32, dense [B][Hq][N] or varlen [Hq][total]; natural
+ *                  log in the scaled-logit domain
+ *   B            : batch size; with cu_seqlens, the number of sequences
+ *   Hq, Hkv      : query / key-value heads; Hq % Hkv == 0.  Query head h
+ *                  reads key/value head h / (Hq / Hkv) (grouped-query
+ *                  attention, "FlashAttention优化" section 5.3, read as
+ *                  contiguous groups)
+ *   N            : sequence length; with cu_seqlens, an upper bound on the
+ *                  longest sequence (sizes the grid; no device->host read)
+ *   d            : head dimension, 64 or 128
+ *   scale        : multiplies Q K^T (normally 1/sqrt(d)), must be > 0
+ *   causal       : nonzero -> key j is masked for query i when j > i
+ *                  (positions counted from the start of each sequence)
+ *   cu_seqlens   : NULL for dense inputs, else device int32[B+1] prefix sums
+ *                  of the sequence lengths (padding-free batches)
+ *   total_tokens : with cu_seqlens, cu_seqlens[B] (the caller's allocation
+ *                  size); ignored for dense inputs
+ *   stream       : CUDA stream the kernels are enqueued on
+ *
+ * Ownership: the caller allocates every buffer (inputs, outputs, and the
+ * backward workspace).  The library allocates no device memory, keeps no
+ * per-call state, and never synchronises the stream.  All pointers are
+ * device pointers and must be 16-byte aligned.
+ *
+ * Errors: argument checks run on the host before any launch and return a
+ * status without touching the device.  A launch failure returns
+ * FA_ERR_CUDA.  Every wait inside the kernels is bounded; a wait that gives
+ * up records a nonzero code that fa_device_error() reports once the caller
+ * has synchronised the stream (the outputs are then undefined).
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad sizes, Hq % Hkv != 0 */
+  FA_ERR_UNSUPPORTED = 2, /* d not in {64, 128} */
+  FA_ERR_WORKSPACE = 3,   /* backward workspace missing or too small */
+  FA_ERR_CUDA = 4         /* a CUDA runtime/driver call or launch failed */
+} fa_status;
+
+/*
+ * Forward: O = softmax(scale Q K^T + mask) V and LSE.
+ * Outputs o (bf16, q's layout) and lse (fp32, layout above) are fully
+ * written for every valid token row; nothing else is touched.
+ * Cites: "注意力机制基础" 2.1 (definition), "FlashAttention优化" 3.1 (tiling),
+ * 3.2.1 (online softmax statistics m and l), paper review 方法 items 1-2
+ * (tiles stay on chip, output rescale by exp(m_old - m_new)).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const int* cu_seqlens, int total_tokens, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: the fp32 row vector
+ * D = rowsum(dO o O) and the fp32 dQ accumulator.  For dense inputs pass
+ * total_tokens = B * N.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens);
+
+/*
+ * Backward by recomputation (paper review, 方法 item 3): P is rebuilt from
+ * Q, K and the forward's LSE; no S or P was stored.  Inputs q, k, v, o, lse,
+ * dO as produced for / by fa_fwd with the same sizes; outputs dq (q's
+ * layout), dk and dv (k's layout; summed over the query heads of each
+ * group).  `workspace` is caller-owned device memory of at least
+ * fa_bwd_workspace_size() bytes, 256-byte aligned; its contents on entry do
+ * not matter.  dQ accumulates in fp32 by atomic addition, so its low bits
+ * may differ between runs; dK and dV are deterministic.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream);
+
+/*
+ * Device-side error word shared by all kernels of the library: 0 when no
+ * wait has timed out since the last fa_clear_device_error().  Reads device
+ * memory synchronously on the current device; call after synchronising.
+ * Returns -1 if the read itself fails.
+ */
+int fa_device_error(void);
+
+/* Reset the device error word to 0 (synchronous). */
+fa_status fa_clear_device_error(void);
+
+/*
+ * Limit, in nanoseconds, for every bounded wait inside the kernels launched
+ * afterwards by this process (default 2e9 = 2 s).  Values below 1000 are
+ * raised to 1000.  Host-side setting only; no device work.
+ */
+void fa_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Diagnostic: launch one CTA that waits on an mbarrier nothing ever arrives
+ * on, with the current wait limit, so that the bounded wait must give up.
+ * It records its code in the error word and returns; the context stays
+ * usable.  Used by the watchdog test.
+ */
+fa_status fa_watchdog_selftest(cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* fa_status_string(fa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,85 @@
+"""C ABI: libfa.so loads, exports every entry point include/fa.h declares, and
+rejects bad arguments on the host before touching the device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_67_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "fa.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"\b(fa_[a-z_]+)\s*\(", txt)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ops.load()
+
+
+def test_header_declares_expected_entry_points():
+    assert set(_declared()) == set(ops.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in ops.STATUS.items():
+        assert ops.fa_status_string(code) == name
+
+
+def _fwd(**kw):
+    a = dict(q=ctypes.c_void_p(4096), k=ctypes.c_void_p(4096), v=ctypes.c_void_p(4096),
+             o=ctypes.c_void_p(4096), lse=ctypes.c_void_p(4096), B=1, Hq=2, Hkv=1, N=128, d=64,
+             scale=0.125, causal=0, cu_seqlens=None, total_tokens=0, stream=None)
+    a.update(kw)
+    return ops.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["N"],
+                      a["d"], a["scale"], a["causal"], a["cu_seqlens"], a["total_tokens"],
+                      a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(d=96), 2), (dict(d=256), 2), (dict(Hq=3, Hkv=2), 1), (dict(Hkv=0), 1),
+    (dict(N=0), 1), (dict(B=-1), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
+    (dict(q=None), 1), (dict(o=ctypes.c_void_p(4100)), 1),
+    (dict(cu_seqlens=ctypes.c_void_p(4096), total_tokens=-1), 1),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, expect):
+    assert _fwd(**kw) == expect
+
+
+def test_fwd_empty_batch_is_a_no_op(lib):
+    # B = 0 and an empty varlen batch need no launch at all
+    assert _fwd(B=0) == 0
+    assert _fwd(cu_seqlens=ctypes.c_void_p(4096), total_tokens=0) == 0
+
+
+def test_bwd_workspace_checks(lib):
+    need = ops.fa_bwd_workspace_size(2, 4, 256, 128, 512)
+    assert need >= 512 * 4 * 128 * 4 + 512 * 4 * 4
+    assert ops.fa_bwd_workspace_size(1, 1, 1, 96, 1) == 0
+    p = ctypes.c_void_p(4096)
+    args = [p] * 9
+    st = ops.fa_bwd(*args, ctypes.c_void_p(4096), need - 1, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
+                    None)
+    assert st == 3
+    st = ops.fa_bwd(*args, None, need, 2, 4, 4, 256, 128, 0.1, 1, None, 0, None)
+    assert st == 3
+    st = ops.fa_bwd(*args, ctypes.c_void_p(4096 + 16), need, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
+                    None)
+    assert st == 3   # workspace must be 256-byte aligned
+
+
+def test_build_command_targets_sm100a():
+    cmd = build.nvcc_command("x.so")
+    assert "arch=compute_100a,code=sm_100a" in cmd
+    assert "-lineinfo" in cmd
