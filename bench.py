@@ -1,0 +1,405 @@
+"""Benchmark: exact attention forward + backward on B200 (TFLOP/s and % of
+dense BF16 tensor peak).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl {b200,reference}] [--no-cpu-baseline] [--no-e2e]
+
+One step = fa_fwd (O, LSE) + fa_bwd (dQ, dK, dV) over one batch of the
+workload, all through the C ABI of libfa.so.  FLOPs: forward 4 B H N^2 d
+(halved for causal), backward 2.5x forward.  Prints ONE JSON line (rank 0).
+
+Multi-GPU (torchrun, one process per GPU): the path partitions into
+independent (sequence, kv-head group) problems, so each rank runs its own
+batch of the same shape (weak scaling) with no data-path collective; the
+host-side barrier and a max-reduction of the elapsed time are the only
+communication.  ``--impl reference`` times the CPU fp64 oracle instead (the
+reference arm; rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("attention fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak")
+DEFAULT_WORKLOAD = "gqa_causal_b2_hq32_hkv8_n4096_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks of the default
+    process group (identity without one).  The only cross-rank traffic of the
+    benchmark besides barriers."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def weak_scaling_value(world_size, flops_per_step_per_rank, steps, ms_max):
+    """Whole-job TFLOP/s: every rank processed `steps` steps of its own batch;
+    the job took as long as the slowest rank."""
+    return world_size * flops_per_step_per_rank * steps / (ms_max / 1e3) / 1e12
+
+
+def rank_workload(w, rank):
+    """Rank r's batch: same shape, its own seed (the ranks hold disjoint
+    independent problems, so nothing is exchanged)."""
+    from exact_io_aware_67_b200 import workloads
+    return workloads.Workload(**{**w.__dict__, "seed": w.seed + rank})
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "") else None,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["power"] is None or r["power"] > 300] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_sample(w, heads, nthreads):
+    """fp64 oracle forward + backward on `heads` (batch, query head) problems of
+    workload w (full sequence length, its causal flag and d), packed as a batch
+    of independent single-head problems.  Returns (seconds, flops)."""
+    import numpy as np
+    import oracle
+    from exact_io_aware_67_b200 import workloads
+    inp = workloads.generate(w)
+    g = w.Hq // w.Hkv
+    qs, ks, vs, ds = [], [], [], []
+    for u in range(heads):
+        b, h = divmod(u, w.Hq)
+        b %= w.B
+        qs.append(inp.q[b, :, h].float().numpy())
+        ks.append(inp.k[b, :, h // g].float().numpy())
+        vs.append(inp.v[b, :, h // g].float().numpy())
+        ds.append(inp.dout[b, :, h].float().numpy())
+    st = lambda a: np.stack(a)[:, :, None, :].astype(np.float64)
+    q, k, v, do = st(qs), st(ks), st(vs), st(ds)
+    t0 = time.perf_counter()
+    oracle.attention_fwd(q, k, v, w.scale, w.causal, nthreads=nthreads)
+    oracle.attention_bwd(q, k, v, do, w.scale, w.causal, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    per_head = 4.0 * w.N * w.N * w.d * (0.5 if w.causal else 1.0)
+    return dt, heads * per_head * 3.5
+
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    cores = len(os.sched_getaffinity(0))
+    heads = max(1, min(cores, 16, w.B * w.Hq))
+    for _ in range(args.warmup):
+        cpu_sample(w, heads, cores)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, f = cpu_sample(w, heads, cores)
+        times.append(dt)
+        flops = f
+    tot = sum(times)
+    value = flops * len(times) / tot / 1e12
+    sample = ("%d (batch, query head) problems of %s per step (N=%d, d=%d, causal=%s), "
+              "fp64 three-pass oracle forward + analytic backward" %
+              (heads, w.name, w.N, w.d, w.causal))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, **w.describe()},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_b200(args, w):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_67_b200 import flops, ops, workloads
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    # each rank draws its own batch of the same shape (weak scaling)
+    wr = rank_workload(w, rank)
+    inp = workloads.generate(wr)
+    lengths = inp.lengths
+    q, k, v, do = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.dout))
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    maxlen = (max(lengths) if lengths else w.N) if cu is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N) if cu is None else (w.Hq, q.shape[0]),
+                      dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_buf = ops.workspace_for(q, k, cu, maxlen)
+    fwd_f = flops.fwd_flops(w, lengths)
+    bwd_f = flops.bwd_flops(w, lengths)
+    step_f = fwd_f + bwd_f
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse)
+        ops.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, cu, maxlen,
+                          workspace=ws_buf, dq=dq, dk=dk, dv=dv)
+
+    ops.fa_clear_device_error()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-kernel events: forward kernel and backward main kernel of every step
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_begin.record(stream)
+    for s in range(args.steps):
+        ops.fa_set_profile_events(ev[s][0], ev[s][1])
+        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse)
+        ops.fa_set_profile_events(ev[s][2], ev[s][3])
+        ops.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, cu, maxlen,
+                          workspace=ws_buf, dq=dq, dk=dk, dv=dv)
+    ops.fa_set_profile_events(None, None)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_begin.elapsed_time(t_end)
+    fwd_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
+    bwd_ms = [ev[s][2].elapsed_time(ev[s][3]) for s in range(args.steps)]
+    err = ops.fa_device_error()
+    if err != 0:
+        raise RuntimeError("device error word 0x%x during the timed region" % err)
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hq = [t.pin_memory() for t in (inp.q, inp.k, inp.v, inp.dout)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in hq)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        for it in range(1 + args.steps):
+            if it == 1:
+                if ws > 1:
+                    dist.barrier()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            for dst, src in zip((q, k, v, do), hq):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(hout, (o, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
+
+    # ---------------------------------------------------------------- reduce
+    ms_max, e2e_max = max_over_ranks([ms, e2e["ms"] if e2e else 0.0], device=dev)
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peaks_src = load_peaks()
+    value = weak_scaling_value(ws, step_f, args.steps, ms_max)
+    fwd_avg = sum(fwd_ms) / len(fwd_ms)
+    bwd_avg = sum(bwd_ms) / len(bwd_ms)
+    fwd_tf = fwd_f / (fwd_avg / 1e3) / 1e12
+    bwd_tf = bwd_f / (bwd_avg / 1e3) / 1e12
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # dominant kernel: the one with the larger share of the step
+    if bwd_avg >= fwd_avg:
+        dom, dom_ms, dom_f = "bwd_main_kernel", bwd_avg, bwd_f
+    else:
+        dom, dom_ms, dom_f = "fwd_kernel", fwd_avg, fwd_f
+    achieved = dom_f / (dom_ms / 1e3) / 1e12
+    traffic = load_traffic(dom, w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 inputs of the workload's shape)",
+        "config": {"workload": w.name, **w.describe(),
+                   "l2": "inputs larger than L2 (%.0f MB touched per step)" %
+                         (bytes_per_step(q, k, v, o, do, dq, dk, dv, ws_buf) / 1e6),
+                   "parallelism": "independent batches per GPU" if ws > 1 else "1 GPU"},
+        "pct_of_peak": 100.0 * value / ws / peak_sus,
+        "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+        "fwd_pct_of_peak": 100.0 * fwd_tf / peak_sus, "bwd_pct_of_peak": 100.0 * bwd_tf / peak_sus,
+        "peak_tflops": peak_sus, "peak_source": "%s bf16_tflops_sustained" % peaks_src,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": achieved / peak_sus,
+                     "frac_of_burst_peak": achieved / peak_burst,
+                     "traffic": traffic,
+                     "algorithmic_flops_per_launch": dom_f, "avg_launch_ms": dom_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = {"value": weak_scaling_value(ws, step_f, args.steps, e2e_max),
+                       "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
+                       "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": e2e_max / args.steps}
+    if not args.no_cpu_baseline and ws == 1:
+        cores = len(os.sched_getaffinity(0))
+        heads = max(1, min(cores, 16, w.B * w.Hq))
+        dt, f = cpu_sample(w, heads, cores)
+        line["cpu_baseline"] = {
+            "value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "seconds": dt,
+            "sample": "%d (batch, query head) problems of the workload (N=%d, d=%d, causal=%s), "
+                      "fp64 oracle forward + backward" % (heads, w.N, w.d, w.causal)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bytes_per_step(*ts):
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if one exists for
+    this kernel and workload and the kernel sources are unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        ent = d.get(kernel, {}).get(workload)
+        if not ent:
+            return None
+        if ent.get("source_sha") != source_sha():
+            return None
+        return ent.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def source_sha():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_67_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    from exact_io_aware_67_b200 import workloads
+    w = workloads.WORKLOADS[args.workload]
+    if args.warmup < 3 and args.impl == "b200":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_b200(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -4,6 +4,8 @@
 // synchronises the caller's stream.
 #include <atomic>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstdint>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -15,6 +17,20 @@
 namespace {
 
 std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+thread_local int t_last_cuda_error = 0;
+// Optional events recorded around the main kernel of the next calls made by
+// this thread (see fa_set_profile_events).
+thread_local cudaEvent_t t_prof_begin = nullptr;
+thread_local cudaEvent_t t_prof_end = nullptr;
+
+// Record a failed CUDA call for fa_last_cuda_error() and map it to a status;
+// with FA_DEBUG set in the environment the failing site is printed.
+fa_status cuda_fail(cudaError_t e, const char* site) {
+  t_last_cuda_error = (int)e;
+  if (std::getenv("FA_DEBUG") != nullptr)
+    std::fprintf(stderr, "libfa: %s failed: %s\n", site, cudaGetErrorString(e));
+  return FA_ERR_CUDA;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
@@ -54,6 +70,26 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int d, int heads, long ro
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Make the device that owns `ptr` current for the calling thread.  A thread
+// that has not touched CUDA yet (autograd's worker, a user thread) has no
+// current context, and tensor-map encoding needs one.  Host pointers are
+// rejected.
+fa_status bind_device_of(const void* ptr) {
+  cudaPointerAttributes a{};
+  cudaError_t e = cudaPointerGetAttributes(&a, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return FA_ERR_INVALID_ARG;
+  // cudaSetDevice also binds the device's primary context to this thread;
+  // cudaGetDevice alone would report device 0 without binding anything.
+  e = cudaSetDevice(a.device);
+  if (e != cudaSuccess) return cuda_fail(e, "select device");
+  return FA_OK;
+}
+
 struct Dims {
   int B, Hq, Hkv, N, d, total;
   bool varlen;
@@ -90,8 +126,11 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)p.num_qblocks * p.Hq * p.B;
+  if (t_prof_begin != nullptr) cudaEventRecord(t_prof_begin, stream);
   kern<<<grid, fa::FWD_THREADS, smem, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess && t_prof_end != nullptr) e = cudaEventRecord(t_prof_end, stream);
+  return e;
 }
 
 }  // namespace
@@ -109,12 +148,14 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
+  st = bind_device_of(q);
+  if (st != FA_OK) return st;
 
   CUtensorMap mq, mk, mv;
   if (!encode_rows_map(&mq, q, d, Hq, s.rows(), s.batches()) ||
       !encode_rows_map(&mk, k, d, Hkv, s.rows(), s.batches()) ||
       !encode_rows_map(&mv, v, d, Hkv, s.rows(), s.batches()))
-    return FA_ERR_CUDA;
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
 
   fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -137,7 +178,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   else
     e = causal ? launch_fwd<128, true>(mq, mk, mv, p, stream)
                : launch_fwd<128, false>(mq, mk, mv, p, stream);
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "forward launch");
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
@@ -162,13 +203,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FA_ERR_WORKSPACE;
+  st = bind_device_of(q);
+  if (st != FA_OK) return st;
 
   CUtensorMap mq, mk, mv, mdo;
   if (!encode_rows_map(&mq, q, d, Hq, s.rows(), s.batches()) ||
       !encode_rows_map(&mk, k, d, Hkv, s.rows(), s.batches()) ||
       !encode_rows_map(&mv, v, d, Hkv, s.rows(), s.batches()) ||
       !encode_rows_map(&mdo, dO, d, Hq, s.rows(), s.batches()))
-    return FA_ERR_CUDA;
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
 
   fa::BwdParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -190,8 +233,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.wait_limit_ns = g_wait_limit_ns.load();
   fa::bwd_carve_workspace(p, workspace, s.tokens(), d);
 
-  const cudaError_t e = fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream);
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t e =
+      fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream, t_prof_begin, t_prof_end);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "backward launch");
 }
 
 int fa_device_error(void) {
@@ -212,7 +256,15 @@ void fa_set_wait_limit_ns(unsigned long long ns) {
 
 fa_status fa_watchdog_selftest(cudaStream_t stream) {
   fa::watchdog_selftest_kernel<<<1, 32, 0, stream>>>(g_wait_limit_ns.load());
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "self-test launch");
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+void fa_set_profile_events(cudaEvent_t main_begin, cudaEvent_t main_end) {
+  t_prof_begin = main_begin;
+  t_prof_end = main_end;
 }
 
 const char* fa_status_string(fa_status s) {

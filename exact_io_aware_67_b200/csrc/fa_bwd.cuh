@@ -1,5 +1,43 @@
-// fa_bwd.cuh -- backward kernels (work in progress: launcher only).
+// fa_bwd.cuh -- backward attention kernels for sm_100a.
+//
+// The backward recomputes S and P from Q, K and the forward's LSE instead of
+// reading stored N x N matrices (paper review "FlashAttention: Fast and
+// Memory-Efficient Exact Attention with IO-Awareness", 方法 item 3).  The
+// gradient formulas are the derivative of O = softmax(scale Q K^T + mask) V:
+//     P = exp(scale S - LSE),  dV = P^T dO,  dP = dO V^T,
+//     D_i = sum_c dO_ic O_ic (= sum_j P_ij dP_ij),  dS = P o (dP - D),
+//     dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels run in stream order:
+//   bwd_pre_kernel     D = rowsum(dO o O) in fp32 and zero the fp32 dQ
+//                      accumulator (HBM-bound, grid-stride).
+//   bwd_main_kernel    one CTA per 128-row K/V tile of one (sequence, kv
+//                      head).  It loops over the query heads of its group and
+//                      over the query tiles (only those on or below the
+//                      diagonal when causal).  dK and dV accumulate in TMEM
+//                      for the whole loop; each tile's dQ partial goes to the
+//                      fp32 accumulator by vector atomic addition.
+//   bwd_dq_kernel      dQ = scale * accumulator -> bf16, transposed back to
+//                      the token-major layout.
+//
+// Orientation in bwd_main_kernel (kv rows are the MMA M dimension, so the
+// per-thread row owned by the elementwise warps is a kv row):
+//   S^T  = K Q^T        SS, A = K (K-major), B = Q (K-major)      -> TMEM
+//   dP^T = V dO^T       SS, A = V (K-major), B = dO (K-major)     -> TMEM
+//   dV  += P^T dO       TS, A = P^T (bf16 in TMEM), B = dO (N-major)
+//   dK  += dS^T Q       SS, A = dS^T (smem, K-major), B = Q (N-major)
+//   dQ_i = dS K         SS, A = dS (same smem, M-major), B = K (N-major)
+// One 128 x 128 bf16 dS tile in shared memory serves both dK and dQ: as
+// [kv row][q] it is K-major for dK and M-major for dQ.
+//
+// dQ accumulator layout (fp32): element (token t, head h, column c) lives at
+//   ((h * d/4 + c/4) * T + t) * 4 + c % 4,   T = token rows of the batch,
+// so the 32 threads of a warp (32 consecutive query rows) add one 512-byte
+// contiguous run per vector atomic.
 #pragma once
+#include <cstdio>
+#include <cstdlib>
+
 #include "fa_common.cuh"
 #include "sm100.cuh"
 
@@ -13,31 +51,591 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  float* dpsum;      // D = rowsum(dO o O), layout of lse
-  float* dq_acc;     // fp32 dQ accumulator
+  float* dpsum;      // D, same layout as lse
+  float* dq_acc;     // fp32 dQ accumulator (layout above)
   const int* cu_seqlens;
   int B, Hq, Hkv, N, group, total;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
 };
 
+inline size_t bwd_dsum_bytes(int Hq, long tokens) {
+  return ((size_t)Hq * (size_t)tokens * 4 + 255) & ~(size_t)255;
+}
+
 inline size_t bwd_workspace_bytes(int Hq, int d, long tokens) {
-  const size_t dsum = ((size_t)Hq * (size_t)tokens * 4 + 255) & ~(size_t)255;
-  const size_t acc = (size_t)tokens * Hq * d * 4;
-  return dsum + acc + 256 * 128;   // slack so the accumulator covers whole tiles
+  return bwd_dsum_bytes(Hq, tokens) + (size_t)tokens * Hq * d * 4;
 }
 
-inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int d) {
+inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int /*d*/) {
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const size_t dsum = ((size_t)p.Hq * (size_t)tokens * 4 + 255) & ~(size_t)255;
   p.dpsum = reinterpret_cast<float*>(base);
-  p.dq_acc = reinterpret_cast<float*>(base + dsum);
-  (void)d;
+  p.dq_acc = reinterpret_cast<float*>(base + bwd_dsum_bytes(p.Hq, tokens));
 }
 
-inline cudaError_t launch_bwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                              const CUtensorMap&, const BwdParams&, int, bool, cudaStream_t) {
-  return cudaErrorNotSupported;
+// statistic index (lse / D) of token row `row` of sequence b, head h
+__device__ __forceinline__ long stat_index(const BwdParams& p, int b, int h, int seq_start,
+                                           int row) {
+  return (p.cu_seqlens != nullptr) ? (long)h * p.total + seq_start + row
+                                   : ((long)b * p.Hq + h) * p.N + row;
+}
+
+// ============================================================================
+// K2: D = rowsum(dO o O) and zeroing of the dQ accumulator
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long tokens) {
+  // zero the accumulator
+  {
+    float4* acc = reinterpret_cast<float4*>(p.dq_acc);
+    const long n4 = tokens * p.Hq * (D / 4);
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
+         i += (long)gridDim.x * blockDim.x)
+      acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // one group of D/8 lanes per (token, head) row; each lane reads 8 bf16
+  constexpr int LPR = D / 8;            // lanes per row
+  constexpr int RPW = 32 / LPR;         // rows per warp pass
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR;
+  const int li = lane % LPR;
+  const long rows = tokens * p.Hq;
+  const long warp_global = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5;
+  const long nwarps = ((long)gridDim.x * blockDim.x) >> 5;
+  for (long base = warp_global * RPW; base < rows; base += nwarps * RPW) {
+    const long row = base + sub;
+    float s = 0.f;
+    if (row < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(p.o + row * D + li * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(p.dout + row * D + li * 8);
+      const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(ah[e]);
+        const float2 y = __bfloat1622float2(bh[e]);
+        s = fmaf(x.x, y.x, s);
+        s = fmaf(x.y, y.y, s);
+      }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (li == 0 && row < rows) {
+      const long t = row / p.Hq;
+      const int h = (int)(row % p.Hq);
+      long idx;
+      if (p.cu_seqlens != nullptr) {
+        idx = (long)h * p.total + t;
+      } else {
+        const long b = t / p.N, n = t % p.N;
+        idx = (b * p.Hq + h) * p.N + n;
+      }
+      p.dpsum[idx] = s;
+    }
+  }
+}
+
+// ============================================================================
+// K4: dQ = scale * accumulator -> bf16 [token][head][d]
+// ============================================================================
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long tokens) {
+  constexpr int TT = 32;                       // tokens per block
+  __shared__ float tile[TT][D + 4];
+  const int h = blockIdx.y;
+  const long t0 = (long)blockIdx.x * TT;
+  for (int idx = threadIdx.x; idx < (D / 4) * TT; idx += blockDim.x) {
+    const int cg = idx / TT, tt = idx % TT;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t0 + tt < tokens)
+      v = reinterpret_cast<const float4*>(p.dq_acc)[((long)h * (D / 4) + cg) * tokens + t0 + tt];
+    tile[tt][4 * cg + 0] = v.x;
+    tile[tt][4 * cg + 1] = v.y;
+    tile[tt][4 * cg + 2] = v.z;
+    tile[tt][4 * cg + 3] = v.w;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < TT * (D / 8); idx += blockDim.x) {
+    const int tt = idx / (D / 8), ch = idx % (D / 8);
+    if (t0 + tt >= tokens) continue;
+    const float* src = &tile[tt][8 * ch];
+    uint4 w;
+    w.x = pack_bf16(src[0] * p.scale, src[1] * p.scale);
+    w.y = pack_bf16(src[2] * p.scale, src[3] * p.scale);
+    w.z = pack_bf16(src[4] * p.scale, src[5] * p.scale);
+    w.w = pack_bf16(src[6] * p.scale, src[7] * p.scale);
+    *reinterpret_cast<uint4*>(p.dq + ((t0 + tt) * p.Hq + h) * D + 8 * ch) = w;
+  }
+}
+
+// ============================================================================
+// K3: main backward kernel
+// ============================================================================
+template <int D>
+struct BwdLayout {
+  static constexpr int TILE = 128 * D * 2;   // one 128 x D bf16 tile
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;            // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;       // 1 stage
+  static constexpr int OFF_DS = OFF_DO + TILE;          // 128 x 128 bf16
+  static constexpr int OFF_STATS = OFF_DS + 32768;      // 2 stages x (lse2[128], D[128])
+  static constexpr int OFF_BAR = OFF_STATS + 2 * 1024;
+  // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
+  // ds_empty dq_full dq_empty dkv_done drain
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+  // TMEM columns
+  static constexpr uint32_t T_DV = 0;
+  static constexpr uint32_t T_DK = D;
+  static constexpr uint32_t T_S = 2 * D;
+  static constexpr uint32_t T_DP = 2 * D + 128;
+  static constexpr uint32_t T_DQ = (D == 128) ? T_DP : 2 * D + 256;   // aliases dP at d = 128
+};
+
+constexpr int BWD_THREADS = 448;   // warps 0-7 elementwise, 8-11 dQ, 12 TMA, 13 MMA
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---------------------------------------------------------------- work item
+  const int nkv_blocks = (p.N + 127) / 128;
+  const int j = (int)(blockIdx.x % nkv_blocks);           // kv tile (low j = most work)
+  const int hk = (int)((blockIdx.x / nkv_blocks) % p.Hkv);
+  const int b = (int)(blockIdx.x / ((unsigned)nkv_blocks * p.Hkv));
+  int seq_start = 0, len = p.N, bcoord = b;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - seq_start;
+    bcoord = 0;
+  }
+  if (128 * j >= len) return;
+  const int nq = (len + 127) / 128;
+  const int i0 = CAUSAL ? j : 0;
+  const int n_i = nq - i0;                  // query tiles per head
+  const int T = p.group * n_i;              // iterations of this CTA
+
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sDO = smem + L::OFF_DO;
+  uint8_t* sDS = smem + L::OFF_DS;
+  float* stats = reinterpret_cast<float*>(smem + L::OFF_STATS);   // [2][2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;      // [2]
+  uint64_t* q_empty = bars + 3;     // [2]
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;
+  uint64_t* s_full = bars + 7;
+  uint64_t* dp_full = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* ds_full = bars + 10;
+  uint64_t* ds_empty = bars + 11;
+  uint64_t* dq_full = bars + 12;
+  uint64_t* dq_empty = bars + 13;
+  uint64_t* dkv_done = bars + 14;
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full + s, 33);   // TMA expect-tx arrival + 32 statistic writers
+      mbar_init(q_empty + s, 1);
+    }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
+    mbar_init(ds_empty, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(dkv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 13) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 12 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
+
+  if (warp == 12) {
+    // ============================================================ producer
+    const float kLog2e = 1.4426950408889634f;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_4d(sK + c * 16384, &tmK, kv_full, c * 64, hk, seq_start + 128 * j, bcoord);
+        tma_load_4d(sV + c * 16384, &tmV, kv_full, c * 64, hk, seq_start + 128 * j, bcoord);
+      }
+    }
+    int q_issued = 0, do_issued = 0;
+    bool ok = true;
+    for (int n = 0; n < T && ok; ++n) {
+      const int h = hk * p.group + n / n_i;
+      const int i = i0 + n % n_i;
+      const int s = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(q_empty + s, ((n >> 1) & 1) ^ 1, wd, ERR_BWD_LOAD_EMPTY));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full + s, L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sQ + s * L::TILE + c * 16384, &tmQ, q_full + s, c * 64, h,
+                      seq_start + 128 * i, bcoord);
+      }
+      q_issued = n + 1;
+      // statistics of the 128 query rows: LSE * log2(e) and D; rows past the
+      // sequence end get +inf / 0 so that their P and dS vanish
+      float* st = stats + s * 256;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = lane + 32 * e;
+        const int row = 128 * i + r;
+        float l2 = INFINITY, dd = 0.f;
+        if (row < len) {
+          const long si = stat_index(p, b, h, seq_start, row);
+          l2 = p.lse[si] * kLog2e;
+          dd = p.dpsum[si];
+        }
+        st[r] = l2;
+        st[128 + r] = dd;
+      }
+      mbar_arrive(q_full + s);
+      ok = __all_sync(0xffffffffu, mbar_wait(do_empty, (n & 1) ^ 1, wd, ERR_BWD_LOAD_EMPTY));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(do_full, L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sDO + c * 16384, &tmDO, do_full, c * 64, h, seq_start + 128 * i, bcoord);
+      }
+      do_issued = n + 1;
+    }
+    if (lane == 0 && *abort_flag) {
+      mbar_wait_drain(kv_full, 0, p.wait_limit_ns);
+      for (int n = max(0, q_issued - 2); n < q_issued; ++n)
+        mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, p.wait_limit_ns);
+      if (do_issued > 0) mbar_wait_drain(do_full, (do_issued - 1) & 1, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_sq = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+      const uint32_t id_kn = idesc_bf16_f32(128, D, false, true);      // dV, dK
+      const uint32_t id_mn = idesc_bf16_f32(128, D, true, true);       // dQ
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ);
+      const uint32_t aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+      // D[128 x 128] = A[128 x D] B[128 x D]^T, both K-major
+      auto mma_nt = [&](uint32_t dcol, uint32_t a, uint32_t bq) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + dcol, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bq + off, 16, 1024),
+                 id_sq, kk > 0);
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, wd, ERR_BWD_KV_FULL);
+      // prologue: S_0 and dP_0
+      if (ok) ok = mbar_wait(q_full + 0, 0, wd, ERR_BWD_Q_FULL);
+      if (ok) {
+        tc_fence_after();
+        mma_nt(L::T_S, aK, aQ);
+        mma_commit(s_full);
+        ok = mbar_wait(do_full, 0, wd, ERR_BWD_Q_FULL);
+      }
+      if (ok) {
+        tc_fence_after();
+        mma_nt(L::T_DP, aV, aDO);
+        mma_commit(dp_full);
+      }
+      for (int n = 0; ok && n < T; ++n) {
+        const int s = n & 1;
+        const uint32_t ph = n & 1;
+        // dV += P^T dO  (A = P^T in TMEM: q columns 0-63 at T_S + 0..31,
+        // 64-127 at T_S + 64..95)
+        if (!(ok = mbar_wait(p_full, ph, wd, ERR_BWD_P_FULL))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acol = L::T_S + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4));
+          mma_ts(tmem + L::T_DV, tmem + acol,
+                 sdesc_sw128(aDO + kk * 2048, 16384, 1024), id_kn, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(do_empty);
+        // dK += dS^T Q  (A = dS^T K-major in smem, B = Q N-major)
+        if (!(ok = mbar_wait(ds_full, ph, wd, ERR_BWD_DS_FULL))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + L::T_DK, sdesc_sw128(aDS + aoff, 16, 1024),
+                 sdesc_sw128(aQ + s * L::TILE + kk * 2048, 16384, 1024), id_kn,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(q_empty + s);
+        // dQ_n = dS K  (A = dS M-major in smem, B = K N-major)
+        if (D != 128 && n > 0) {
+          if (!(ok = mbar_wait(dq_empty, (n - 1) & 1, wd, ERR_BWD_DQ_EMPTY))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::T_DQ, sdesc_sw128(aDS + kk * 2048, 16384, 1024),
+                 sdesc_sw128(aK + kk * 2048, 16384, 1024), id_mn, kk > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        mma_commit(ds_empty);
+        if (n + 1 < T) {
+          const int s1 = (n + 1) & 1;
+          if (!(ok = mbar_wait(q_full + s1, ((n + 1) >> 1) & 1, wd, ERR_BWD_Q_FULL))) break;
+          tc_fence_after();
+          mma_nt(L::T_S, aK, aQ + s1 * L::TILE);
+          mma_commit(s_full);
+          if (!(ok = mbar_wait(do_full, (n + 1) & 1, wd, ERR_BWD_Q_FULL))) break;
+          if (D == 128) {
+            // the dP columns still hold dQ_n until the dQ warps have read it
+            if (!(ok = mbar_wait(dq_empty, n & 1, wd, ERR_BWD_DQ_EMPTY))) break;
+          }
+          tc_fence_after();
+          mma_nt(L::T_DP, aV, aDO);
+          mma_commit(dp_full);
+        }
+      }
+      mma_commit(dkv_done);
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // ============================================================ dQ drain
+    const int r = (warp & 3) * 32 + lane;                 // query row within tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tq = tmem + lane_off + L::T_DQ;
+    const long Ttok = (p.cu_seqlens != nullptr) ? (long)p.total : (long)p.B * p.N;
+    for (int n = 0; n < T; ++n) {
+      const int h = hk * p.group + n / n_i;
+      const int i = i0 + n % n_i;
+      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, n & 1, wd, ERR_BWD_DQ_FULL))) break;
+      tc_fence_after();
+      const int row = 128 * i + r;
+      const bool row_ok = row < len;
+      const long t = (p.cu_seqlens != nullptr) ? (long)seq_start + row : (long)b * p.N + row;
+      float4* acc = reinterpret_cast<float4*>(p.dq_acc) + (long)h * (D / 4) * Ttok + t;
+#pragma unroll
+      for (int half = 0; half < D / 64; ++half) {
+        uint32_t v[64];
+        tmem_ld32(tq + half * 64, v);
+        tmem_ld32(tq + half * 64 + 32, v + 32);
+        tmem_wait_ld32(v);
+        tmem_wait_ld32(v + 32);
+        if (half == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int g4 = 0; g4 < 16; ++g4)
+            atomicAdd(acc + (long)(half * 16 + g4) * Ttok,
+                      make_float4(__uint_as_float(v[4 * g4]), __uint_as_float(v[4 * g4 + 1]),
+                                  __uint_as_float(v[4 * g4 + 2]), __uint_as_float(v[4 * g4 + 3])));
+        }
+      }
+    }
+  } else {
+    // ============================================================ elementwise
+    // warp w owns kv rows 32 (w % 4) .. +31 (its TMEM lanes); warpgroup
+    // wg = w / 4 owns query columns 64 wg .. 64 wg + 63 of the tile.
+    const int wg = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;                 // kv row within tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + L::T_S + 64 * wg;
+    const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * wg;
+    const int kv_row = 128 * j + r;
+    const bool kv_ok = kv_row < len;
+    const float c2 = p.scale_log2;
+    // byte offset of this thread's row inside its 64-column dS region
+    uint8_t* ds_row = sDS + wg * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+    bool ok = true;
+    for (int n = 0; n < T; ++n) {
+      const int i = i0 + n % n_i;
+      const int s = n & 1;
+      const float* st = stats + s * 256;
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, wd, ERR_BWD_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      float P[64];
+      {
+        uint32_t sv[64];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tS + 32, sv + 32);
+        tmem_wait_ld32(sv);
+        tmem_wait_ld32(sv + 32);
+        // causal diagonal tile: key row kv_row is masked for query q < kv_row
+        const int qlim = (CAUSAL && i == j) ? (kv_row - 128 * i - 64 * wg) : 0;
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(st + 64 * wg + 4 * c4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * c4 + e;
+            float pv = ex2(fmaf(__uint_as_float(sv[c]), c2, -lv[e]));
+            if (!kv_ok || c < qlim) pv = 0.f;
+            P[c] = pv;
+          }
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(P[2 * c], P[2 * c + 1]);
+        tmem_st32(tS, pk);      // P^T (bf16) over the S columns just read
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(p_full);
+      // dS = P o (dP - D)
+      ok = __all_sync(0xffffffffu, mbar_wait(dp_full, n & 1, wd, ERR_BWD_DP_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dsp[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dv[32];
+        tmem_ld32(tDP + 32 * hh, dv);
+        tmem_wait_ld32(dv);
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(st + 128 + 64 * wg + 32 * hh + 4 * c4);
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+          float ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 32 * hh + 4 * c4 + e;
+            ds[e] = P[c] * (__uint_as_float(dv[4 * c4 + e]) - dd[e]);
+          }
+          dsp[16 * hh + 2 * c4] = pack_bf16(ds[0], ds[1]);
+          dsp[16 * hh + 2 * c4 + 1] = pack_bf16(ds[2], ds[3]);
+        }
+      }
+      // the previous dS tile must have been consumed by its dK and dQ products
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(ds_empty, (n - 1) & 1, wd, ERR_BWD_DS_FULL));
+        if (!ok) break;
+      }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const int pos = ch ^ (r & 7);       // 128-byte swizzle
+        *reinterpret_cast<uint4*>(ds_row + pos * 16) =
+            make_uint4(dsp[4 * ch], dsp[4 * ch + 1], dsp[4 * ch + 2], dsp[4 * ch + 3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_done, 0, wd, ERR_BWD_DKV_DONE));
+    if (ok) {
+      tc_fence_after();
+      const uint32_t tcol = tmem + lane_off + (wg == 0 ? L::T_DV : L::T_DK);
+      const float mul = (wg == 0) ? 1.f : p.scale;
+      __nv_bfloat16* dst = (wg == 0) ? p.dv : p.dk;
+      const long t = (p.cu_seqlens != nullptr) ? (long)seq_start + kv_row : (long)b * p.N + kv_row;
+      __nv_bfloat16* row_ptr = dst + (t * p.Hkv + hk) * (long)D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tcol + 32 * c, v);
+        tmem_wait_ld32(v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        if (kv_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(row_ptr + 32 * c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mdo, const BwdParams& p, cudaStream_t stream,
+                         cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+  const long tokens = (p.cu_seqlens != nullptr) ? (long)p.total : (long)p.B * p.N;
+  bwd_pre_kernel<D><<<148 * 8, 256, 0, stream>>>(p, tokens);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: pre kernel launch\n");
+    return e;
+  }
+  auto kern = bwd_main_kernel<D, CAUSAL>;
+  const int smem = BwdLayout<D>::ALLOC;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) {
+    if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: set smem attribute\n");
+    return e;
+  }
+  const unsigned grid = (unsigned)((p.N + 127) / 128) * p.Hkv * p.B;
+  if (ev_begin != nullptr) cudaEventRecord(ev_begin, stream);
+  kern<<<grid, BWD_THREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && ev_end != nullptr) e = cudaEventRecord(ev_end, stream);
+  if (e != cudaSuccess) {
+    if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: main kernel launch\n");
+    return e;
+  }
+  dim3 g2((unsigned)((tokens + 31) / 32), (unsigned)p.Hq);
+  bwd_dq_kernel<D><<<g2, 256, 0, stream>>>(p, tokens);
+  return cudaGetLastError();
+}
+
+inline cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                              const CUtensorMap& mdo, const BwdParams& p, int d, bool causal,
+                              cudaStream_t stream, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+  if (d == 64)
+    return causal ? launch_bwd_t<64, true>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
+                  : launch_bwd_t<64, false>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
+  return causal ? launch_bwd_t<128, true>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
+                : launch_bwd_t<128, false>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
 }
 
 // One warp waits on an mbarrier that nothing arrives on; the bounded wait

@@ -23,12 +23,15 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
-            "fa_status_string"]
+            "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events"]
 
 
 class FAError(RuntimeError):
     def __init__(self, fn, status):
-        super().__init__("%s failed: %s" % (fn, STATUS.get(status, status)))
+        msg = "%s failed: %s" % (fn, STATUS.get(status, status))
+        if status == 4:
+            msg += " (cudaError %d)" % fa_last_cuda_error()
+        super().__init__(msg)
         self.status = status
 
 
@@ -64,6 +67,10 @@ def load(build_if_missing=True):
     lib.fa_set_wait_limit_ns.restype = None
     lib.fa_watchdog_selftest.argtypes = [vp]
     lib.fa_watchdog_selftest.restype = c_int
+    lib.fa_set_profile_events.argtypes = [vp, vp]
+    lib.fa_set_profile_events.restype = None
+    lib.fa_last_cuda_error.argtypes = []
+    lib.fa_last_cuda_error.restype = c_int
     lib.fa_status_string.argtypes = [c_int]
     lib.fa_status_string.restype = ctypes.c_char_p
     if os.environ.get("FA_WAIT_LIMIT_NS"):
@@ -103,6 +110,17 @@ def fa_set_wait_limit_ns(ns):
 
 def fa_watchdog_selftest(stream):
     return load().fa_watchdog_selftest(stream)
+
+
+def fa_set_profile_events(main_begin, main_end):
+    """main_begin / main_end: torch.cuda.Event objects (or None to stop)."""
+    b = None if main_begin is None else ctypes.c_void_p(main_begin.cuda_event)
+    e = None if main_end is None else ctypes.c_void_p(main_end.cuda_event)
+    load().fa_set_profile_events(b, e)
+
+
+def fa_last_cuda_error():
+    return load().fa_last_cuda_error()
 
 
 def fa_status_string(s):

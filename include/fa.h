@@ -40,7 +40,10 @@
  * Ownership: the caller allocates every buffer (inputs, outputs, and the
  * backward workspace).  The library allocates no device memory, keeps no
  * per-call state, and never synchronises the stream.  All pointers are
- * device pointers and must be 16-byte aligned.
+ * device pointers on one device and must be 16-byte aligned.  The kernels
+ * run on the device that owns q: if it is not the calling thread's current
+ * device, the call makes it current (this also gives a thread that has not
+ * used CUDA before a context).  A host pointer for q is FA_ERR_INVALID_ARG.
  *
  * Errors: argument checks run on the host before any launch and return a
  * status without touching the device.  A launch failure returns
@@ -125,6 +128,22 @@ void fa_set_wait_limit_ns(unsigned long long ns);
  * usable.  Used by the watchdog test.
  */
 fa_status fa_watchdog_selftest(cudaStream_t stream);
+
+/*
+ * The cudaError_t value behind the most recent FA_ERR_CUDA returned to the
+ * calling thread (0 if none).  Host-side, thread-local; no device work.
+ */
+int fa_last_cuda_error(void);
+
+/*
+ * Instrumentation: when main_begin / main_end are non-NULL, every later
+ * fa_fwd / fa_bwd call made by this thread records them on its stream right
+ * before and right after its main kernel (the attention kernel itself, not
+ * the backward's pre- and post-processing kernels), so that the caller can
+ * time that kernel with cudaEventElapsedTime.  Pass NULL, NULL to stop.  The
+ * events stay owned by the caller.  Host-side setting only.
+ */
+void fa_set_profile_events(cudaEvent_t main_begin, cudaEvent_t main_end);
 
 /* Human-readable name of a status code (static storage). */
 const char* fa_status_string(fa_status s);
