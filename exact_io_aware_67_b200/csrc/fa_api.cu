@@ -183,7 +183,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
   if (B < 0 || Hq < 1 || N < 1 || (d != 64 && d != 128) || total_tokens < 0) return 0;
-  return fa::bwd_workspace_bytes(Hq, d, (long)total_tokens);
+  // the size must serve a dense call (total_tokens = B * N) and a varlen
+  // call with the same numbers, so take the larger of the two layouts
+  const size_t a = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, false);
+  const size_t v = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, true);
+  return a > v ? a : v;
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -199,7 +203,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
-  const size_t need = fa::bwd_workspace_bytes(Hq, d, s.tokens());
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d, s.tokens(), s.varlen);
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FA_ERR_WORKSPACE;

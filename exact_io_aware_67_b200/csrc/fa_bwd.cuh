@@ -30,10 +30,17 @@
 // One 128 x 128 bf16 dS tile in shared memory serves both dK and dQ: as
 // [kv row][q] it is K-major for dK and M-major for dQ.
 //
-// dQ accumulator layout (fp32): element (token t, head h, column c) lives at
-//   ((h * d/4 + c/4) * T + t) * 4 + c % 4,   T = token rows of the batch,
-// so the 32 threads of a warp (32 consecutive query rows) add one 512-byte
-// contiguous run per vector atomic.
+// dQ accumulator layout (fp32, tile-major): query tile i of sequence b has
+// its own 128-row block at tile slot  tb(b) + i,  where
+//   tb(b) = b * ceil(N / 128)                 (dense batches)
+//   tb(b) = ceil(cu_seqlens[b] / 128) + b     (variable-length batches),
+// which never overlaps the next sequence's slots.  Inside a slot the layout
+// is [head][column group of 4][row 0..127][4], so the 32 threads of a warp
+// (32 consecutive rows) add one contiguous 512-byte run per vector atomic.
+// Rows of a tile past the end of its sequence are never added and never read.
+// (Measured alternative: staging the tile in shared memory and adding it with
+// bulk asynchronous reductions was slower -- the reductions from one issuing
+// thread proceed nearly one after another.)
 #pragma once
 #include <cstdio>
 #include <cstdlib>
@@ -53,6 +60,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   float* dpsum;      // D, same layout as lse
   float* dq_acc;     // fp32 dQ accumulator (layout above)
+  long tile_slots;   // tile slots of the accumulator per head
   const int* cu_seqlens;
   int B, Hq, Hkv, N, group, total;
   float scale, scale_log2;
@@ -63,14 +71,32 @@ inline size_t bwd_dsum_bytes(int Hq, long tokens) {
   return ((size_t)Hq * (size_t)tokens * 4 + 255) & ~(size_t)255;
 }
 
-inline size_t bwd_workspace_bytes(int Hq, int d, long tokens) {
-  return bwd_dsum_bytes(Hq, tokens) + (size_t)tokens * Hq * d * 4;
+// number of 128-row tile slots of the dQ accumulator
+inline long bwd_tile_slots(int B, int N, long tokens, bool varlen) {
+  return varlen ? (tokens + 127) / 128 + B : (long)B * ((N + 127) / 128);
+}
+
+inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d, long tokens, bool varlen) {
+  return bwd_dsum_bytes(Hq, tokens) + (size_t)bwd_tile_slots(B, N, tokens, varlen) * Hq * 128 * d * 4;
 }
 
 inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int /*d*/) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   p.dpsum = reinterpret_cast<float*>(base);
   p.dq_acc = reinterpret_cast<float*>(base + bwd_dsum_bytes(p.Hq, tokens));
+  p.tile_slots = bwd_tile_slots(p.B, p.N, tokens, p.cu_seqlens != nullptr);
+}
+
+// first tile slot of sequence b
+__device__ __forceinline__ long tile_base(const BwdParams& p, int b) {
+  return (p.cu_seqlens != nullptr) ? (long)((p.cu_seqlens[b] + 127) / 128) + b
+                                   : (long)b * ((p.N + 127) / 128);
+}
+
+// fp32 offset of (head h, tile slot ts, column group 0, row 0)
+template <int D>
+__device__ __forceinline__ long acc_tile_offset(const BwdParams& p, int h, long ts) {
+  return ((long)h * p.tile_slots + ts) * (long)(128 * D);
 }
 
 // statistic index (lse / D) of token row `row` of sequence b, head h
@@ -88,7 +114,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long to
   // zero the accumulator
   {
     float4* acc = reinterpret_cast<float4*>(p.dq_acc);
-    const long n4 = tokens * p.Hq * (D / 4);
+    const long n4 = p.tile_slots * p.Hq * 128 * (D / 4);
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
          i += (long)gridDim.x * blockDim.x)
       acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -138,33 +164,45 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long to
 // ============================================================================
 // K4: dQ = scale * accumulator -> bf16 [token][head][d]
 // ============================================================================
+// grid: (query tiles of the longest sequence, Hq, B); 256 threads; each block
+// turns one 128-row tile (two halves of 64 rows) back into token-major bf16.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long tokens) {
-  constexpr int TT = 32;                       // tokens per block
-  __shared__ float tile[TT][D + 4];
-  const int h = blockIdx.y;
-  const long t0 = (long)blockIdx.x * TT;
-  for (int idx = threadIdx.x; idx < (D / 4) * TT; idx += blockDim.x) {
-    const int cg = idx / TT, tt = idx % TT;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (t0 + tt < tokens)
-      v = reinterpret_cast<const float4*>(p.dq_acc)[((long)h * (D / 4) + cg) * tokens + t0 + tt];
-    tile[tt][4 * cg + 0] = v.x;
-    tile[tt][4 * cg + 1] = v.y;
-    tile[tt][4 * cg + 2] = v.z;
-    tile[tt][4 * cg + 3] = v.w;
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
+  constexpr int RH = 64;                       // rows per half
+  __shared__ float tile[RH][D + 4];
+  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  int seq_start = 0, len = p.N;
+  if (p.cu_seqlens != nullptr) {
+    seq_start = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - seq_start;
   }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < TT * (D / 8); idx += blockDim.x) {
-    const int tt = idx / (D / 8), ch = idx % (D / 8);
-    if (t0 + tt >= tokens) continue;
-    const float* src = &tile[tt][8 * ch];
-    uint4 w;
-    w.x = pack_bf16(src[0] * p.scale, src[1] * p.scale);
-    w.y = pack_bf16(src[2] * p.scale, src[3] * p.scale);
-    w.z = pack_bf16(src[4] * p.scale, src[5] * p.scale);
-    w.w = pack_bf16(src[6] * p.scale, src[7] * p.scale);
-    *reinterpret_cast<uint4*>(p.dq + ((t0 + tt) * p.Hq + h) * D + 8 * ch) = w;
+  if (128 * i >= len) return;
+  const long tok0 = ((p.cu_seqlens != nullptr) ? (long)seq_start : (long)b * p.N) + 128 * i;
+  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + acc_tile_offset<D>(p, h, tile_base(p, b) + i));
+  for (int half = 0; half < 2; ++half) {
+    const int r0 = half * RH;
+    if (128 * i + r0 >= len) break;
+    for (int idx = threadIdx.x; idx < (D / 4) * RH; idx += blockDim.x) {
+      const int cg = idx / RH, rr = idx % RH;
+      const float4 v = src[cg * 128 + r0 + rr];
+      tile[rr][4 * cg + 0] = v.x;
+      tile[rr][4 * cg + 1] = v.y;
+      tile[rr][4 * cg + 2] = v.z;
+      tile[rr][4 * cg + 3] = v.w;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < RH * (D / 8); idx += blockDim.x) {
+      const int rr = idx / (D / 8), ch = idx % (D / 8);
+      if (128 * i + r0 + rr >= len) continue;
+      const float* f = &tile[rr][8 * ch];
+      uint4 w;
+      w.x = pack_bf16(f[0] * p.scale, f[1] * p.scale);
+      w.y = pack_bf16(f[2] * p.scale, f[3] * p.scale);
+      w.z = pack_bf16(f[4] * p.scale, f[5] * p.scale);
+      w.w = pack_bf16(f[6] * p.scale, f[7] * p.scale);
+      *reinterpret_cast<uint4*>(p.dq + ((tok0 + r0 + rr) * p.Hq + h) * D + 8 * ch) = w;
+    }
+    __syncthreads();
   }
 }
 
@@ -176,17 +214,22 @@ struct BwdLayout {
   static constexpr int TILE = 128 * D * 2;   // one 128 x D bf16 tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int DO_STAGES = 2;
   static constexpr int OFF_Q = OFF_V + TILE;            // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * TILE;       // 1 stage
-  static constexpr int OFF_DS = OFF_DO + TILE;          // 128 x 128 bf16
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;       // DO_STAGES stages
+  static constexpr int OFF_DS = OFF_DO + DO_STAGES * TILE;   // 128 x 128 bf16
   static constexpr int OFF_STATS = OFF_DS + 32768;      // 2 stages x (lse2[128], D[128])
   static constexpr int OFF_BAR = OFF_STATS + 2 * 1024;
-  // kv_full q_full[2] q_empty[2] do_full do_empty s_full dp_full p_full ds_full
-  // ds_empty dq_full dq_empty dkv_done drain
-  static constexpr int NBAR = 16;
+  // kv_full q_full[2] q_empty[2] st_full[2] do_full[2] do_empty[2] s_full dp_full
+  // p_full ds_full ds_empty dq_full dq_empty dkv_done drain
+  static constexpr int NBAR = 20;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;
+  // The d = 128 layout uses all but ~0.8 KB of the 227 KB a CTA may have, so
+  // it relies on the dynamic shared memory window starting 1024-byte aligned
+  // (checked at run time; a misaligned base reports ERR_BWD_SMEM_ALIGN).
+  static constexpr bool SLACK = (BYTES + 1024 <= 232448);
+  static constexpr int ALLOC = SLACK ? BYTES + 1024 : BYTES;
   // TMEM columns
   static constexpr uint32_t T_DV = 0;
   static constexpr uint32_t T_DK = D;
@@ -195,7 +238,13 @@ struct BwdLayout {
   static constexpr uint32_t T_DQ = (D == 128) ? T_DP : 2 * D + 256;   // aliases dP at d = 128
 };
 
-constexpr int BWD_THREADS = 448;   // warps 0-7 elementwise, 8-11 dQ, 12 TMA, 13 MMA
+// warps 0-7: elementwise (two warpgroups, 64 query columns each)
+// warps 8-11: dQ drain;  warp 12: TMA producer;  warp 13: MMA issuer;
+// warps 14-15: idle (they only give their registers to the drain warps)
+constexpr int BWD_THREADS = 512;
+constexpr int BWD_REGS_DRAIN = 176;   // warpgroup 2 after setmaxnreg.inc
+constexpr int BWD_REGS_CTRL = 80;     // warpgroup 3 after setmaxnreg.dec
+static_assert(128 * (128 + 128 + BWD_REGS_DRAIN + BWD_REGS_CTRL) == 65536, "register split");
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
@@ -204,9 +253,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                     const BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (!L::SLACK && (smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicCAS(&g_fa_error, 0, ERR_BWD_SMEM_ALIGN);
+    return;
+  }
+  uint8_t* smem = L::SLACK ? align_1024(smem_raw) : smem_raw;
 
   // ---------------------------------------------------------------- work item
   const int nkv_blocks = (p.N + 127) / 128;
@@ -235,28 +288,30 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;      // [2]
   uint64_t* q_empty = bars + 3;     // [2]
-  uint64_t* do_full = bars + 5;
-  uint64_t* do_empty = bars + 6;
-  uint64_t* s_full = bars + 7;
-  uint64_t* dp_full = bars + 8;
-  uint64_t* p_full = bars + 9;
-  uint64_t* ds_full = bars + 10;
-  uint64_t* ds_empty = bars + 11;
-  uint64_t* dq_full = bars + 12;
-  uint64_t* dq_empty = bars + 13;
-  uint64_t* dkv_done = bars + 14;
-  uint64_t* drain = bars + 15;
+  uint64_t* st_full = bars + 5;     // [2]  statistics of the Q stage
+  uint64_t* do_full = bars + 7;     // [2]
+  uint64_t* do_empty = bars + 9;    // [2]
+  uint64_t* s_full = bars + 11;
+  uint64_t* dp_full = bars + 12;
+  uint64_t* p_full = bars + 13;
+  uint64_t* ds_full = bars + 14;
+  uint64_t* ds_empty = bars + 15;
+  uint64_t* dq_full = bars + 16;
+  uint64_t* dq_empty = bars + 17;
+  uint64_t* dkv_done = bars + 18;
+  uint64_t* drain = bars + 19;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(q_full + s, 33);   // TMA expect-tx arrival + 32 statistic writers
+      mbar_init(q_full + s, 1);
       mbar_init(q_empty + s, 1);
+      mbar_init(st_full + s, 32);
+      mbar_init(do_full + s, 1);
+      mbar_init(do_empty + s, 1);
     }
-    mbar_init(do_full, 1);
-    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
@@ -285,6 +340,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
 
+  if (warp >= 12) {
+  // ============================================================== warpgroup 3
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(BWD_REGS_CTRL));
   if (warp == 12) {
     // ============================================================ producer
     const float kLog2e = 1.4426950408889634f;
@@ -302,7 +360,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int h = hk * p.group + n / n_i;
       const int i = i0 + n % n_i;
       const int s = n & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(q_empty + s, ((n >> 1) & 1) ^ 1, wd, ERR_BWD_LOAD_EMPTY));
+      const uint32_t ph_empty = ((n >> 1) & 1) ^ 1;
+      // Q_n (stage s) and dO_n (stage s) by TMA
+      ok = __all_sync(0xffffffffu, mbar_wait(q_empty + s, ph_empty, wd, ERR_BWD_LOAD_EMPTY));
       if (!ok) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(q_full + s, L::TILE);
@@ -312,55 +372,71 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                       seq_start + 128 * i, bcoord);
       }
       q_issued = n + 1;
+      const int sd = n % L::DO_STAGES;
+      ok = __all_sync(0xffffffffu, mbar_wait(do_empty + sd, ((n / L::DO_STAGES) & 1) ^ 1, wd,
+                                             ERR_BWD_LOAD_EMPTY));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(do_full + sd, L::TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(sDO + sd * L::TILE + c * 16384, &tmDO, do_full + sd, c * 64, h,
+                      seq_start + 128 * i, bcoord);
+      }
+      do_issued = n + 1;
       // statistics of the 128 query rows: LSE * log2(e) and D; rows past the
-      // sequence end get +inf / 0 so that their P and dS vanish
+      // sequence end get +inf / 0 so that their P and dS vanish.  The stage's
+      // previous readers are done: they finished before dK of iteration n-2,
+      // which released q_empty[s].
+      float lv[4], dv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = 128 * i + lane + 32 * e;
+        const long si = stat_index(p, b, h, seq_start, min(row, len - 1));
+        lv[e] = p.lse[si];
+        dv[e] = p.dpsum[si];
+      }
       float* st = stats + s * 256;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = lane + 32 * e;
-        const int row = 128 * i + r;
-        float l2 = INFINITY, dd = 0.f;
-        if (row < len) {
-          const long si = stat_index(p, b, h, seq_start, row);
-          l2 = p.lse[si] * kLog2e;
-          dd = p.dpsum[si];
-        }
-        st[r] = l2;
-        st[128 + r] = dd;
+        const bool valid = 128 * i + r < len;
+        st[r] = valid ? lv[e] * kLog2e : INFINITY;
+        st[128 + r] = valid ? dv[e] : 0.f;
       }
-      mbar_arrive(q_full + s);
-      ok = __all_sync(0xffffffffu, mbar_wait(do_empty, (n & 1) ^ 1, wd, ERR_BWD_LOAD_EMPTY));
-      if (!ok) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(do_full, L::TILE);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sDO + c * 16384, &tmDO, do_full, c * 64, h, seq_start + 128 * i, bcoord);
-      }
-      do_issued = n + 1;
+      mbar_arrive(st_full + s);
     }
     if (lane == 0 && *abort_flag) {
       mbar_wait_drain(kv_full, 0, p.wait_limit_ns);
       for (int n = max(0, q_issued - 2); n < q_issued; ++n)
         mbar_wait_drain(q_full + (n & 1), (n >> 1) & 1, p.wait_limit_ns);
-      if (do_issued > 0) mbar_wait_drain(do_full, (do_issued - 1) & 1, p.wait_limit_ns);
+      for (int n = max(0, do_issued - L::DO_STAGES); n < do_issued; ++n)
+        mbar_wait_drain(do_full + n % L::DO_STAGES, (n / L::DO_STAGES) & 1, p.wait_limit_ns);
     }
     __syncwarp();
   } else if (warp == 13) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      const uint32_t id_sq = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-      const uint32_t id_kn = idesc_bf16_f32(128, D, false, true);      // dV, dK
-      const uint32_t id_mn = idesc_bf16_f32(128, D, true, true);       // dQ
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ);
-      const uint32_t aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+      constexpr uint32_t id_sq = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t id_kn = idesc_bf16_f32(128, D, false, true);      // dV, dK
+      constexpr uint32_t id_mn = idesc_bf16_f32(128, D, true, true);       // dQ
+      // descriptors built once; K-major views (LBO unused) and N/M-major
+      // views (LBO = distance between 64-element blocks)
+      const SDesc kK = sdesc_make(smem_u32(sK), 16, 1024);     // K, A of S^T
+      const SDesc kV = sdesc_make(smem_u32(sV), 16, 1024);     // V, A of dP^T
+      const SDesc kQ = sdesc_make(smem_u32(sQ), 16, 1024);     // Q, B of S^T
+      const SDesc kDO = sdesc_make(smem_u32(sDO), 16, 1024);   // dO, B of dP^T
+      const SDesc kDS = sdesc_make(smem_u32(sDS), 16, 1024);   // dS^T, A of dK
+      const SDesc nDO = sdesc_make(smem_u32(sDO), 16384, 1024);  // dO, B of dV
+      const SDesc nQ = sdesc_make(smem_u32(sQ), 16384, 1024);    // Q, B of dK
+      const SDesc nK = sdesc_make(smem_u32(sK), 16384, 1024);    // K, B of dQ
+      const SDesc mDS = sdesc_make(smem_u32(sDS), 16384, 1024);  // dS, A of dQ
       // D[128 x 128] = A[128 x D] B[128 x D]^T, both K-major
-      auto mma_nt = [&](uint32_t dcol, uint32_t a, uint32_t bq) {
+      auto mma_nt = [&](uint32_t dcol, SDesc a, SDesc bq, uint32_t boff) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + dcol, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bq + off, 16, 1024),
-                 id_sq, kk > 0);
+          mma_ss(tmem + dcol, sdesc_at(a, off), sdesc_at(bq, boff + off), id_sq, kk > 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(kv_full, 0, wd, ERR_BWD_KV_FULL);
@@ -368,18 +444,24 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (ok) ok = mbar_wait(q_full + 0, 0, wd, ERR_BWD_Q_FULL);
       if (ok) {
         tc_fence_after();
-        mma_nt(L::T_S, aK, aQ);
+        mma_nt(L::T_S, kK, kQ, 0);
         mma_commit(s_full);
-        ok = mbar_wait(do_full, 0, wd, ERR_BWD_Q_FULL);
+        ok = mbar_wait(do_full + 0, 0, wd, ERR_BWD_Q_FULL);
       }
       if (ok) {
         tc_fence_after();
-        mma_nt(L::T_DP, aV, aDO);
+        mma_nt(L::T_DP, kV, kDO, 0);
         mma_commit(dp_full);
       }
+      // Steady state, iteration n (issue order; the tensor pipe runs them in
+      // this order):  dV_n, S_{n+1}, dQ_n, dK_n, dP_{n+1}.  S_{n+1} goes out
+      // right after the last reader of P_n so that the elementwise warps can
+      // build P_{n+1} while dQ_n and dK_n run; dQ_n precedes dK_n so that its
+      // TMEM drain overlaps dK_n.
       for (int n = 0; ok && n < T; ++n) {
         const int s = n & 1;
         const uint32_t ph = n & 1;
+        const bool has_next = n + 1 < T;
         // dV += P^T dO  (A = P^T in TMEM: q columns 0-63 at T_S + 0..31,
         // 64-127 at T_S + 64..95)
         if (!(ok = mbar_wait(p_full, ph, wd, ERR_BWD_P_FULL))) break;
@@ -388,20 +470,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t acol = L::T_S + (kk < 4 ? 8 * kk : 64 + 8 * (kk - 4));
           mma_ts(tmem + L::T_DV, tmem + acol,
-                 sdesc_sw128(aDO + kk * 2048, 16384, 1024), id_kn, (n > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(do_empty);
-        // dK += dS^T Q  (A = dS^T K-major in smem, B = Q N-major)
-        if (!(ok = mbar_wait(ds_full, ph, wd, ERR_BWD_DS_FULL))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + L::T_DK, sdesc_sw128(aDS + aoff, 16, 1024),
-                 sdesc_sw128(aQ + s * L::TILE + kk * 2048, 16384, 1024), id_kn,
+                 sdesc_at(nDO, (n % L::DO_STAGES) * L::TILE + kk * 2048), id_kn,
                  (n > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(q_empty + s);
+        mma_commit(do_empty + n % L::DO_STAGES);
+        if (has_next) {
+          const int s1 = (n + 1) & 1;
+          if (!(ok = mbar_wait(q_full + s1, ((n + 1) >> 1) & 1, wd, ERR_BWD_Q_FULL))) break;
+          tc_fence_after();
+          mma_nt(L::T_S, kK, kQ, s1 * L::TILE);
+          mma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, ph, wd, ERR_BWD_DS_FULL))) break;
+        tc_fence_after();
         // dQ_n = dS K  (A = dS M-major in smem, B = K N-major)
         if (D != 128 && n > 0) {
           if (!(ok = mbar_wait(dq_empty, (n - 1) & 1, wd, ERR_BWD_DQ_EMPTY))) break;
@@ -409,23 +490,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + L::T_DQ, sdesc_sw128(aDS + kk * 2048, 16384, 1024),
-                 sdesc_sw128(aK + kk * 2048, 16384, 1024), id_mn, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + L::T_DQ, sdesc_at(mDS, kk * 2048), sdesc_at(nK, kk * 2048), id_mn,
+                 kk > 0 ? 1u : 0u);
         mma_commit(dq_full);
+        // dK += dS^T Q  (A = dS^T K-major in smem, B = Q N-major)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + L::T_DK, sdesc_at(kDS, aoff), sdesc_at(nQ, s * L::TILE + kk * 2048), id_kn,
+                 (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(q_empty + s);
         mma_commit(ds_empty);
-        if (n + 1 < T) {
-          const int s1 = (n + 1) & 1;
-          if (!(ok = mbar_wait(q_full + s1, ((n + 1) >> 1) & 1, wd, ERR_BWD_Q_FULL))) break;
-          tc_fence_after();
-          mma_nt(L::T_S, aK, aQ + s1 * L::TILE);
-          mma_commit(s_full);
-          if (!(ok = mbar_wait(do_full, (n + 1) & 1, wd, ERR_BWD_Q_FULL))) break;
+        if (has_next) {
+          const int sd1 = (n + 1) % L::DO_STAGES;
+          if (!(ok = mbar_wait(do_full + sd1, ((n + 1) / L::DO_STAGES) & 1, wd, ERR_BWD_Q_FULL)))
+            break;
           if (D == 128) {
-            // the dP columns still hold dQ_n until the dQ warps have read it
+            // the dP columns hold dQ_n until the dQ warps have read it
             if (!(ok = mbar_wait(dq_empty, n & 1, wd, ERR_BWD_DQ_EMPTY))) break;
           }
           tc_fence_after();
-          mma_nt(L::T_DP, aV, aDO);
+          mma_nt(L::T_DP, kV, kDO, sd1 * L::TILE);
           mma_commit(dp_full);
         }
       }
@@ -434,39 +520,39 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_wait_drain(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else if (warp >= 8) {
     // ============================================================ dQ drain
-    const int r = (warp & 3) * 32 + lane;                 // query row within tile
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(BWD_REGS_DRAIN));
+    // Each thread owns one query row of the tile (its TMEM lane).  The whole
+    // row is read out of TMEM first so the columns can be released early;
+    // then the row is added into the fp32 accumulator with vector atomics.
+    // In the tile-major accumulator the 32 lanes of a warp cover 32
+    // consecutive rows of one column group: one 512-byte run per instruction.
+    const int r = (warp & 3) * 32 + lane;                  // query row within tile
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tq = tmem + lane_off + L::T_DQ;
-    const long Ttok = (p.cu_seqlens != nullptr) ? (long)p.total : (long)p.B * p.N;
+    const long tb = tile_base(p, b);
     for (int n = 0; n < T; ++n) {
       const int h = hk * p.group + n / n_i;
       const int i = i0 + n % n_i;
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, n & 1, wd, ERR_BWD_DQ_FULL))) break;
       tc_fence_after();
-      const int row = 128 * i + r;
-      const bool row_ok = row < len;
-      const long t = (p.cu_seqlens != nullptr) ? (long)seq_start + row : (long)b * p.N + row;
-      float4* acc = reinterpret_cast<float4*>(p.dq_acc) + (long)h * (D / 4) * Ttok + t;
+      uint32_t v[D];
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
-        uint32_t v[64];
-        tmem_ld32(tq + half * 64, v);
-        tmem_ld32(tq + half * 64 + 32, v + 32);
-        tmem_wait_ld32(v);
-        tmem_wait_ld32(v + 32);
-        if (half == D / 64 - 1) {
-          tc_fence_before();
-          mbar_arrive(dq_empty);
-        }
-        if (row_ok) {
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tq + 32 * c, v + 32 * c);
 #pragma unroll
-          for (int g4 = 0; g4 < 16; ++g4)
-            atomicAdd(acc + (long)(half * 16 + g4) * Ttok,
-                      make_float4(__uint_as_float(v[4 * g4]), __uint_as_float(v[4 * g4 + 1]),
-                                  __uint_as_float(v[4 * g4 + 2]), __uint_as_float(v[4 * g4 + 3])));
-        }
+      for (int c = 0; c < D / 32; ++c) tmem_wait_ld32(v + 32 * c);
+      tc_fence_before();
+      mbar_arrive(dq_empty);
+      // rows past the end of the sequence hold exact zeros: skip them
+      if (128 * i + r < len) {
+        float4* acc = reinterpret_cast<float4*>(p.dq_acc + acc_tile_offset<D>(p, h, tb + i)) + r;
+#pragma unroll
+        for (int g = 0; g < D / 4; ++g)
+          atomicAdd(acc + g * 128, make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                               __uint_as_float(v[4 * g + 2]),
+                                               __uint_as_float(v[4 * g + 3])));
       }
     }
   } else {
@@ -488,7 +574,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int i = i0 + n % n_i;
       const int s = n & 1;
       const float* st = stats + s * 256;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, wd, ERR_BWD_S_FULL));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, wd, ERR_BWD_S_FULL) &&
+                                       mbar_wait(st_full + s, (n >> 1) & 1, wd, ERR_BWD_STATS));
       if (!ok) break;
       tc_fence_after();
       float P[64];
@@ -498,19 +585,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_ld32(tS + 32, sv + 32);
         tmem_wait_ld32(sv);
         tmem_wait_ld32(sv + 32);
-        // causal diagonal tile: key row kv_row is masked for query q < kv_row
-        const int qlim = (CAUSAL && i == j) ? (kv_row - 128 * i - 64 * wg) : 0;
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
           const float4 l4 = *reinterpret_cast<const float4*>(st + 64 * wg + 4 * c4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          P[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), c2, -l4.x));
+          P[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), c2, -l4.y));
+          P[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), c2, -l4.z));
+          P[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), c2, -l4.w));
+        }
+        // masks (warp-uniform test first): causal diagonal tile -- key row
+        // kv_row is masked for query q < kv_row -- and key rows past the end
+        // of the sequence
+        const bool diag = CAUSAL && i == j;
+        if (__any_sync(0xffffffffu, diag || !kv_ok)) {
+          const int qlim = diag ? (kv_row - 128 * i - 64 * wg) : 0;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * c4 + e;
-            float pv = ex2(fmaf(__uint_as_float(sv[c]), c2, -lv[e]));
-            if (!kv_ok || c < qlim) pv = 0.f;
-            P[c] = pv;
-          }
+          for (int c = 0; c < 64; ++c)
+            if (!kv_ok || c < qlim) P[c] = 0.f;
         }
         uint32_t pk[32];
 #pragma unroll
@@ -623,8 +714,8 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: main kernel launch\n");
     return e;
   }
-  dim3 g2((unsigned)((tokens + 31) / 32), (unsigned)p.Hq);
-  bwd_dq_kernel<D><<<g2, 256, 0, stream>>>(p, tokens);
+  dim3 g2((unsigned)((p.N + 127) / 128), (unsigned)p.Hq, (unsigned)p.B);
+  bwd_dq_kernel<D><<<g2, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

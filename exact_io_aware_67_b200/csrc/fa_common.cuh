@@ -28,6 +28,7 @@ enum : int {
   ERR_BWD_DKV_DONE = 0x209,
   ERR_BWD_DP_FULL = 0x20a,
   ERR_BWD_STATS = 0x20b,
+  ERR_BWD_SMEM_ALIGN = 0x20c,
   ERR_SELFTEST = 0x301,
 };
 

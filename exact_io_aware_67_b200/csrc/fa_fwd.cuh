@@ -166,28 +166,32 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   } else if (warp == 9) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t ring_addr = smem_u32(ring);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      // descriptors built once: Q tiles and the ring, K-major view (S) and
+      // N-major view (V as the B operand of PV)
+      const SDesc dq = sdesc_make(smem_u32(sQ), 16, 1024);
+      const SDesc dk = sdesc_make(smem_u32(ring), 16, 1024);
+      const SDesc dv = sdesc_make(smem_u32(ring), 16384, 1024);
       // S_t = Q_t K^T : A = Q_t (K-major), B = K tile (K-major), K-dim = d
       auto issue_s = [&](int t, int stage) {
         const uint32_t dt = tmem + t * 128;
+        const uint32_t qo = t * L::TILE, ko = stage * L::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(dt, sdesc_sw128(q_addr + t * L::TILE + off, 16, 1024),
-                 sdesc_sw128(ring_addr + stage * L::TILE + off, 16, 1024), idesc_s, kk > 0);
+          mma_ss(dt, sdesc_at(dq, qo + off), sdesc_at(dk, ko + off), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       // O_t (+)= P_t V : A = P_t from TMEM, B = V tile (N = d contiguous)
       auto issue_pv = [&](int t, int stage, bool acc) {
         const uint32_t dt = tmem + 256 + t * D;
         const uint32_t at = tmem + t * 128;
+        const uint32_t vo = stage * L::TILE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dt, at + kk * 8, sdesc_sw128(ring_addr + stage * L::TILE + kk * 2048, 16384, 1024),
-                 idesc_o, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(dt, at + kk * 8, sdesc_at(dv, vo + kk * 2048), idesc_o,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)

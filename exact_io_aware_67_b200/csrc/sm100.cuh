@@ -151,6 +151,25 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// A descriptor split into its two 32-bit words.  The issuing thread builds
+// one per operand tile up front; advancing to a K-step, a stage or a second
+// 64-element block only adds (byte offset >> 4) to the low word, so each MMA
+// costs one integer add per operand instead of a full descriptor build.
+// (The start-address field is 14 bits of (address >> 4); shared memory stays
+// below 256 KB, so the add never carries out of the field.)
+struct SDesc {
+  uint32_t lo, hi;
+};
+
+__device__ __forceinline__ SDesc sdesc_make(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  const uint64_t d = sdesc_sw128(saddr, lbo, sbo);
+  return SDesc{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+
+__device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t byte_offset) {
+  return ((uint64_t)d.hi << 32) | (uint64_t)(d.lo + (byte_offset >> 4));
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T  (issued by one thread)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {

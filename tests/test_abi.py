@@ -69,7 +69,7 @@ def test_bwd_workspace_checks(lib):
     assert ops.fa_bwd_workspace_size(1, 1, 1, 96, 1) == 0
     p = ctypes.c_void_p(4096)
     args = [p] * 9
-    st = ops.fa_bwd(*args, ctypes.c_void_p(4096), need - 1, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
+    st = ops.fa_bwd(*args, ctypes.c_void_p(4096), 1024, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
                     None)
     assert st == 3
     st = ops.fa_bwd(*args, None, need, 2, 4, 4, 256, 128, 0.1, 1, None, 0, None)
