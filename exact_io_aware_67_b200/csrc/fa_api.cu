@@ -133,6 +133,32 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return e;
 }
 
+// Fixed scratch for fa_bwd_noalloc(): file-scope device memory, so that
+// callers who cannot allocate still get a working backward.  In host code
+// this name is only a stand-in for the symbol; its device address comes
+// from cudaGetSymbolAddress, looked up once per device and cached.
+static __device__ __align__(256) unsigned char g_fa_bwd_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+
+// Device address of g_fa_bwd_scratch on the current device (nullptr and a
+// recorded error on failure).
+void* scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* ptr = g_scratch_addr[dev].load();
+  if (ptr == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_fa_bwd_scratch);
+    if (e != cudaSuccess) {
+      cuda_fail(e, "scratch symbol address");
+      return nullptr;
+    }
+    g_scratch_addr[dev].store(ptr);
+  }
+  return ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -240,6 +266,26 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   const cudaError_t e =
       fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream, t_prof_begin, t_prof_end);
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "backward launch");
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                         int Hq, int Hkv, int N, int d, float scale, int causal,
+                         const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
+  const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
+  bool empty = false;
+  fa_status st = check_dims(s, scale, &empty);
+  if (st != FA_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d, s.tokens(), s.varlen);
+  if (need > (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  st = bind_device_of(q);
+  if (st != FA_OK) return st;
+  void* scratch = scratch_on_current_device();
+  if (scratch == nullptr) return FA_ERR_CUDA;
+  return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Hq, Hkv,
+                N, d, scale, causal, cu_seqlens, total_tokens, stream);
 }
 
 int fa_device_error(void) {

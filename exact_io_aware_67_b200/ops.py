@@ -23,7 +23,11 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
-            "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events"]
+            "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events",
+            "fa_bwd_noalloc"]
+
+# capacity of the fixed scratch behind fa_bwd_noalloc (include/fa.h)
+FA_BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class FAError(RuntimeError):
@@ -57,6 +61,8 @@ def load(build_if_missing=True):
     lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t] + [c_int] * 5 + \
         [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd.restype = c_int
+    lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
+    lib.fa_bwd_noalloc.restype = c_int
     lib.fa_bwd_workspace_size.argtypes = [c_int] * 5
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_device_error.argtypes = []
@@ -90,6 +96,14 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, H
            scale, causal, cu_seqlens, total_tokens, stream):
     return load().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq,
                          Hkv, N, d, scale, int(causal), cu_seqlens, total_tokens, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, cu_seqlens,
+                   total_tokens, stream):
+    """Backward through the library's fixed scratch array (no allocation by
+    the library or by this binding); see include/fa.h for its limits."""
+    return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
+                                 int(causal), cu_seqlens, total_tokens, stream)
 
 
 def fa_bwd_workspace_size(B, Hq, N, d, total_tokens):

@@ -104,6 +104,41 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
 /*
+ * Capacity, in bytes, of the fixed scratch array behind fa_bwd_noalloc().
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * Backward without any allocation -- an addition of this library; the pages
+ * have no counterpart.  Same arguments, layouts and results as fa_bwd(),
+ * minus the workspace: the scratch lives in one fixed 64 MiB array of
+ * device memory inside the library (FA_BWD_NOALLOC_SCRATCH_BYTES), which
+ * every GPU that loads the library holds until the process exits.
+ *
+ * For callers that cannot allocate device memory at call time -- for
+ * example code running under a memory pool or allocator it must not
+ * bypass, a runtime that forbids cudaMalloc/cudaFree on the hot path, or a
+ * host that has no allocator of its own to hand the library.  This entry
+ * point calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Limits and behaviour:
+ *  - If the problem needs more scratch than the fixed capacity (compare
+ *    fa_bwd_workspace_size() with FA_BWD_NOALLOC_SCRATCH_BYTES), the call
+ *    returns FA_ERR_WORKSPACE before launching anything.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last
+ *    call's contents; each call re-initialises what it needs.  Calls whose
+ *    kernels overlap on the GPU (different streams, no ordering between
+ *    them) race on the array and give wrong results: serialise them.
+ */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
+                         int Hq, int Hkv, int N, int d, float scale, int causal,
+                         const int* cu_seqlens, int total_tokens, cudaStream_t stream);
+
+/*
  * Device-side error word shared by all kernels of the library: 0 when no
  * wait has timed out since the last fa_clear_device_error().  Reads device
  * memory synchronously on the current device; call after synchronising.
