@@ -50,8 +50,21 @@ struct FwdLayout {
   static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
 };
 
-constexpr int FWD_THREADS = 320;   // warps 0-7 softmax, 8 TMA, 9 MMA
+// warps 0-7: softmax (two warpgroups); warp 8: TMA; warp 9: MMA; warps 10-11
+// only give their registers to the softmax warpgroups
+constexpr int FWD_THREADS = 384;
+constexpr int FWD_REGS_SOFTMAX = 216;   // warpgroups 0-1 after setmaxnreg.inc
+constexpr int FWD_REGS_CTRL = 72;       // warpgroup 2 after setmaxnreg.dec
+static_assert(128 * (2 * FWD_REGS_SOFTMAX + FWD_REGS_CTRL) <= 65536 &&
+                  2 * (FWD_REGS_SOFTMAX - 168) * 128 == (168 - FWD_REGS_CTRL) * 128,
+              "register split");
 constexpr float RESCALE_LOG2 = 8.0f;
+// Pairs out of every 8 column pairs whose exp2 runs on the FMA pipe
+// (ex2_poly) instead of MUFU.  Measured on B200: with one softmax warp per
+// sub-partition the exp phase is MUFU-bound at ~10 cycles per warp-wide exp2,
+// and moving 2 or 3 pairs in 8 to the FMA pipe made that warp slower (its
+// in-order issue cannot hide the polynomial's dependency chain), so 0.
+constexpr int EXP2_POLY_PAIRS_OF_8 = 0;
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
@@ -130,6 +143,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
 
+  if (warp >= 8) {
+  // ============================================================== warpgroup 2
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(FWD_REGS_CTRL));
   if (warp == 8) {
     // ============================================================ TMA producer
     if (lane == 0) {
@@ -246,8 +262,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       mbar_wait_drain(drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else {
     // ============================================================ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(FWD_REGS_SOFTMAX));
     const int t = warp >> 2;
     const int r = (warp & 3) * 32 + lane;                 // row in tile == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -266,30 +284,36 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       uint32_t s[128];
       tmem_ld32(tS + 0, s + 0);
       tmem_ld32(tS + 32, s + 32);
-      tmem_ld32(tS + 64, s + 64);
-      tmem_ld32(tS + 96, s + 96);
       tmem_wait_ld32(s + 0);
       tmem_wait_ld32(s + 32);
-      tmem_wait_ld32(s + 64);
-      tmem_wait_ld32(s + 96);
-      if (j == n - 1) {
-        // last tile of this Q tile: sequence end and/or causal diagonal
-        int lim = len - 128 * j;
-        if (CAUSAL) lim = min(lim, qrow + 1 - 128 * j);
+      tmem_ld32(tS + 64, s + 64);      // second half loads while the first half is scanned
+      tmem_ld32(tS + 96, s + 96);
+      // last tile of this Q tile: sequence end and/or causal diagonal mask
+      const bool masked = (j == n - 1);
+      int lim = len - 128 * j;
+      if (CAUSAL) lim = min(lim, qrow + 1 - 128 * j);
+      if (masked) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= lim) s[c] = 0xff800000u;   // -inf
       }
-      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+      // row max: four independent chains of 3-input max
+      float mx[4] = {__uint_as_float(s[0]), __uint_as_float(s[1]), __uint_as_float(s[2]),
+                     __uint_as_float(s[3])};
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c + 0]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      for (int c = 4; c < 64; c += 2)
+        mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      tmem_wait_ld32(s + 64);
+      tmem_wait_ld32(s + 96);
+      if (masked) {
+#pragma unroll
+        for (int c = 64; c < 128; ++c)
+          if (c >= lim) s[c] = 0xff800000u;
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c2;
+#pragma unroll
+      for (int c = 64; c < 128; c += 2)
+        mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c2;
       float alpha = 1.f;
       bool resc = false;
       if (m_tile > m + RESCALE_LOG2) {
@@ -299,21 +323,36 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       }
       l *= alpha;
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float l0 = 0.f, l1 = 0.f;
+      // p = 2^(x - m); EXP2_POLY_PAIRS_OF_8 pairs in every 8 use the FMA-pipe
+      // exp2, the rest MUFU
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(s[32 * cc + 2 * i]), c2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(s[32 * cc + 2 * i + 1]), c2, neg_m));
-          l0 += p0;
-          l1 += p1;
+          const float x0 = fmaf(__uint_as_float(s[32 * cc + 2 * i]), c2, neg_m);
+          const float x1 = fmaf(__uint_as_float(s[32 * cc + 2 * i + 1]), c2, neg_m);
+          float p0, p1;
+          if ((i & 7) >= 8 - EXP2_POLY_PAIRS_OF_8) {
+            p0 = ex2_poly(x0);
+            p1 = ex2_poly(x1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          if (i & 1) {
+            l2 += p0;
+            l3 += p1;
+          } else {
+            l0 += p0;
+            l1 += p1;
+          }
           pk[i] = pack_bf16(p0, p1);
         }
         tmem_st16(tS + 16 * cc, pk);
       }
-      l += l0 + l1;
+      l += (l0 + l1) + (l2 + l3);
       tmem_wait_st();
       if (__any_sync(0xffffffffu, resc)) {
         // O_t holds PV of all earlier tiles (S_t of this tile was issued

@@ -273,6 +273,31 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 2^7 (used for part of a row's exponentials so
+// that the MUFU unit is not the only source).  Range reduction: n = round(x)
+// via the 1.5 * 2^23 rounding constant, f = x - n in [-1/2, 1/2]; 2^f by a
+// cubic whose coefficients minimise the maximum relative error on [-1/2, 1/2]
+// (Remez exchange, exact_io_aware_67_b200/fit_exp2.py: 7.5e-5); 2^n is added
+// to the exponent field.  x is clamped at -125 so the result stays a normal
+// number; below that the true value (< 2^-125) is far under any bf16 or
+// fp32-sum resolution that matters here.
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;            // round(x) lands in t's low mantissa bits
+  const float f = x - (t - 12582912.f);      // f in [-1/2, 1/2]
+  float p = fmaf(f, 5.517166853e-02f, 2.426111251e-01f);
+  p = fmaf(p, f, 6.932609677e-01f);
+  p = fmaf(p, f, 9.999280572e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// max of three
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
