@@ -17,6 +17,8 @@ enum : int {
   ERR_FWD_P_FULL = 0x104,
   ERR_FWD_S_FULL = 0x105,
   ERR_FWD_O_DONE = 0x106,
+  ERR_FWD_S_FREE = 0x107,
+  ERR_FWD_P_FREE = 0x108,
   ERR_BWD_LOAD_EMPTY = 0x201,
   ERR_BWD_KV_FULL = 0x202,
   ERR_BWD_Q_FULL = 0x203,

@@ -15,8 +15,16 @@
 //    tile 0, the MMA warp runs tile 1's products and vice versa.
 //  * S = Q K^T and O += P V run as tcgen05.mma (M = 128) with fp32
 //    accumulators in TMEM: S_t at columns [128 t, 128 t + 128), O_t at
-//    [256 + d t, 256 + d t + d).  P (bf16) overwrites the first 64 columns of
-//    S_t and feeds the PV product straight from TMEM.
+//    [256 + d t, 256 + d t + d).  Where P (bf16) lives depends on d:
+//      d = 128: P overwrites the first 64 columns of S_t and feeds PV from
+//               TMEM (TS MMA).  Keeping P out of shared memory matters here:
+//               with P in shared memory the tensor core's operand reads, the
+//               TMA fills and the P stores need ~384 KB per K/V tile, about
+//               3k cycles of shared-memory bandwidth against 2k of MMA work.
+//      d = 64:  P goes to its own 128B-swizzled shared-memory tile, so S_t's
+//               columns are free as soon as the softmax has read them; the
+//               MMA warp issues the next S_t at once and the softmax (the
+//               bottleneck at d = 64, bound by MUFU exp2) never waits for PV.
 //  * One TMA warp fills a ring of K/V stages (mbarrier full/empty pairs),
 //    one thread issues all MMAs, and each softmax warpgroup owns one Q tile:
 //    a thread owns one query row (TMEM lane), so row max and row sum are
@@ -42,9 +50,11 @@ struct FwdLayout {
   static constexpr int NS = (D == 128) ? 3 : 6;  // K/V ring stages
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = 2 * TILE;
-  static constexpr int OFF_BAR = OFF_RING + NS * TILE;
-  // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2] o_done[2] drain[1]
-  static constexpr int NBAR = 2 + 2 * NS + 7;
+  static constexpr bool P_SMEM = (D == 64);             // where P lives (see above)
+  static constexpr int OFF_P = OFF_RING + NS * TILE;    // 2 x 128 x 128 bf16 if P_SMEM
+  static constexpr int OFF_BAR = OFF_P + (P_SMEM ? 2 * 32768 : 0);
+  // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] s_free[2] p_full[2] p_free[2] drain[1]
+  static constexpr int NBAR = 2 + 2 * NS + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
@@ -106,10 +116,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* s_full = kv_empty + NS;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 2;
+  uint64_t* s_full = kv_empty + NS;   // S_t in TMEM (MMA commit)
+  uint64_t* s_free = s_full + 2;      // S_t read out by the softmax (128 threads)
+  uint64_t* p_full = s_free + 2;      // P_t written, O_t rescaled (128 threads)
+  uint64_t* p_free = p_full + 2;      // PV_t done: P_t buffer free, O_t current (commit)
+  uint64_t* drain = p_free + 2;
+  uint8_t* sP = smem + L::OFF_P;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -117,8 +129,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(q_full + i, 1);
       mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 128);
       mbar_init(p_full + i, 128);
-      mbar_init(o_done + i, 1);
+      mbar_init(p_free + i, 1);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full + s, 1);
@@ -184,11 +197,12 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      // descriptors built once: Q tiles and the ring, K-major view (S) and
-      // N-major view (V as the B operand of PV)
+      // descriptors built once: Q tiles, the ring (K-major view for S, N-major
+      // view for V as the B operand of PV) and the P tiles (K-major)
       const SDesc dq = sdesc_make(smem_u32(sQ), 16, 1024);
       const SDesc dk = sdesc_make(smem_u32(ring), 16, 1024);
       const SDesc dv = sdesc_make(smem_u32(ring), 16384, 1024);
+      const SDesc dp = sdesc_make(smem_u32(sP), 16, 1024);
       // S_t = Q_t K^T : A = Q_t (K-major), B = K tile (K-major), K-dim = d
       auto issue_s = [&](int t, int stage) {
         const uint32_t dt = tmem + t * 128;
@@ -199,15 +213,24 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           mma_ss(dt, sdesc_at(dq, qo + off), sdesc_at(dk, ko + off), idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t (+)= P_t V : A = P_t from TMEM, B = V tile (N = d contiguous)
+      // O_t (+)= P_t V : A = P_t (TMEM, or smem K-major), B = V tile (N = d
+      // contiguous)
       auto issue_pv = [&](int t, int stage, bool acc) {
         const uint32_t dt = tmem + 256 + t * D;
-        const uint32_t at = tmem + t * 128;
         const uint32_t vo = stage * L::TILE;
+        if constexpr (L::P_SMEM) {
+          const uint32_t po = t * 32768;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(dt, at + kk * 8, sdesc_at(dv, vo + kk * 2048), idesc_o,
-                 (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(dt, sdesc_at(dp, po + (kk >> 2) * 16384 + (kk & 3) * 32),
+                   sdesc_at(dv, vo + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
+        } else {
+          const uint32_t at = tmem + t * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(dt, at + kk * 8, sdesc_at(dv, vo + kk * 2048), idesc_o,
+                   (acc || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
@@ -222,39 +245,75 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           }
         mma_commit(kv_empty + 0);
       }
-      for (int j = 0; ok && j < nmax; ++j) {
-        const int nv = 2 * j + 1, sv = nv % NS;
-        const int nk = 2 * j + 2, sk = nk % NS;
-        const bool has_next = j + 1 < nmax;
-        if (!(ok = mbar_wait(kv_full + sv, (nv / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
-        tc_fence_after();
-        if (j < n_t[0]) {
-          if (!(ok = mbar_wait(p_full + 0, j & 1, wd, ERR_FWD_P_FULL))) break;
-          tc_fence_after();
-          issue_pv(0, sv, j > 0);
-          if (j == n_t[0] - 1) mma_commit(o_done + 0);
-        }
-        if (has_next) {
-          if (!(ok = mbar_wait(kv_full + sk, (nk / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
-          tc_fence_after();
-          if (j + 1 < n_t[0]) {
-            issue_s(0, sk);
-            mma_commit(s_full + 0);
+      if constexpr (L::P_SMEM) {
+        // Per K/V tile j and Q tile t: S_t of tile j+1 as soon as the softmax
+        // has read S_t^j, then PV_t^j once P_t^j is in shared memory.
+        for (int j = 0; ok && j < nmax; ++j) {
+          const int nv = 2 * j + 1, sv = nv % NS;
+          const int nk = 2 * j + 2, sk = nk % NS;
+          const bool has_next = j + 1 < nmax;
+          if (has_next) {
+            if (!(ok = mbar_wait(kv_full + sk, (nk / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
+            tc_fence_after();
           }
-        }
-        if (j < n_t[1]) {
-          if (!(ok = mbar_wait(p_full + 1, j & 1, wd, ERR_FWD_P_FULL))) break;
+          if (!(ok = mbar_wait(kv_full + sv, (nv / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
           tc_fence_after();
-          issue_pv(1, sv, j > 0);
-          if (j == n_t[1] - 1) mma_commit(o_done + 1);
-        }
-        mma_commit(kv_empty + sv);
-        if (has_next) {
-          if (j + 1 < n_t[1]) {
-            issue_s(1, sk);
-            mma_commit(s_full + 1);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (has_next && j + 1 < n_t[t]) {
+              if (!(ok = mbar_wait(s_free + t, j & 1, wd, ERR_FWD_S_FREE))) break;
+              tc_fence_after();
+              issue_s(t, sk);
+              mma_commit(s_full + t);
+            }
+            if (j < n_t[t]) {
+              if (!(ok = mbar_wait(p_full + t, j & 1, wd, ERR_FWD_P_FULL))) break;
+              tc_fence_after();
+              issue_pv(t, sv, j > 0);
+              mma_commit(p_free + t);
+            }
           }
-          mma_commit(kv_empty + sk);
+          if (!ok) break;
+          if (has_next) mma_commit(kv_empty + sk);
+          mma_commit(kv_empty + sv);
+        }
+      } else {
+        // P aliases S_t, so S_t of tile j+1 follows PV_t^j; the two Q tiles
+        // ping-pong: PV_0^j, S_0^{j+1}, PV_1^j, S_1^{j+1}.
+        for (int j = 0; ok && j < nmax; ++j) {
+          const int nv = 2 * j + 1, sv = nv % NS;
+          const int nk = 2 * j + 2, sk = nk % NS;
+          const bool has_next = j + 1 < nmax;
+          if (!(ok = mbar_wait(kv_full + sv, (nv / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
+          tc_fence_after();
+          if (j < n_t[0]) {
+            if (!(ok = mbar_wait(p_full + 0, j & 1, wd, ERR_FWD_P_FULL))) break;
+            tc_fence_after();
+            issue_pv(0, sv, j > 0);
+            mma_commit(p_free + 0);
+          }
+          if (has_next) {
+            if (!(ok = mbar_wait(kv_full + sk, (nk / NS) & 1, wd, ERR_FWD_KV_FULL))) break;
+            tc_fence_after();
+            if (j + 1 < n_t[0]) {
+              issue_s(0, sk);
+              mma_commit(s_full + 0);
+            }
+          }
+          if (j < n_t[1]) {
+            if (!(ok = mbar_wait(p_full + 1, j & 1, wd, ERR_FWD_P_FULL))) break;
+            tc_fence_after();
+            issue_pv(1, sv, j > 0);
+            mma_commit(p_free + 1);
+          }
+          mma_commit(kv_empty + sv);
+          if (has_next) {
+            if (j + 1 < n_t[1]) {
+              issue_s(1, sk);
+              mma_commit(s_full + 1);
+            }
+            mma_commit(kv_empty + sk);
+          }
         }
       }
       // every MMA issued above completes before TMEM can be released
@@ -305,6 +364,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
       tmem_wait_ld32(s + 64);
       tmem_wait_ld32(s + 96);
+      // S_t is in registers: the MMA warp may compute the next S_t now
+      tc_fence_before();
+      mbar_arrive(s_free + t);
       if (masked) {
 #pragma unroll
         for (int c = 64; c < 128; ++c)
@@ -323,8 +385,30 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       }
       l *= alpha;
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      if (L::P_SMEM && j > 0) {
+        // PV_t of the previous K/V tile must be done: it reads the P_t buffer
+        // and accumulates into O_t.  (With P in TMEM, S_t^j was issued after
+        // that PV, so s_full already implies it.)
+        ok = __all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, wd, ERR_FWD_P_FREE));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld32(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
       // p = 2^(x - m); EXP2_POLY_PAIRS_OF_8 pairs in every 8 use the FMA-pipe
-      // exp2, the rest MUFU
+      // exp2, the rest MUFU.  P (bf16) goes to this row of the 128B-swizzled
+      // K-major P tile: columns 0-63 and 64-127 are two 16 KB regions.
+      uint8_t* prow = sP + (L::P_SMEM ? t * 32768 + (r >> 3) * 1024 + (r & 7) * 128 : 0);
       float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -350,30 +434,29 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           }
           pk[i] = pack_bf16(p0, p1);
         }
-        tmem_st16(tS + 16 * cc, pk);
+        if constexpr (L::P_SMEM) {
+          uint8_t* reg = prow + (cc >> 1) * 16384;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int ch = (cc & 1) * 4 + k;
+            *reinterpret_cast<uint4*>(reg + ((ch ^ (r & 7)) * 16)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
+        } else {
+          tmem_st16(tS + 16 * cc, pk);   // P_t over the S_t columns already read
+        }
       }
       l += (l0 + l1) + (l2 + l3);
-      tmem_wait_st();
-      if (__any_sync(0xffffffffu, resc)) {
-        // O_t holds PV of all earlier tiles (S_t of this tile was issued
-        // after them), so it can be rescaled in place now.
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld32(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
+      if constexpr (L::P_SMEM)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      else
         tmem_wait_st();
-      }
       tc_fence_before();
       mbar_arrive(p_full + t);
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_done + t, 0, wd, ERR_FWD_O_DONE));
+      ok = __all_sync(0xffffffffu, mbar_wait(p_free + t, (n - 1) & 1, wd, ERR_FWD_O_DONE));
       if (ok) {
         tc_fence_after();
         const bool row_ok = qrow < len;
