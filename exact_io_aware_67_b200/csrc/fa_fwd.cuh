@@ -70,10 +70,13 @@ static_assert(128 * (2 * FWD_REGS_SOFTMAX + FWD_REGS_CTRL) <= 65536 &&
               "register split");
 constexpr float RESCALE_LOG2 = 8.0f;
 // Pairs out of every 8 column pairs whose exp2 runs on the FMA pipe
-// (ex2_poly) instead of MUFU.  Measured on B200: with one softmax warp per
-// sub-partition the exp phase is MUFU-bound at ~10 cycles per warp-wide exp2,
-// and moving 2 or 3 pairs in 8 to the FMA pipe made that warp slower (its
-// in-order issue cannot hide the polynomial's dependency chain), so 0.
+// (ex2_poly) instead of MUFU.  Measured on B200 (forward TFLOP/s, causal
+// H=16 N=16384 d=64): 0 -> 716, 2 -> 651, 3 -> 606, 4 -> 565, and slower at
+// d=128 too: the scalar cubic costs more issue slots than the MUFU time it
+// frees, so 0.  (Taking the exponentials against the running max before the
+// tile's max is known, redoing the rare tile whose max moved, was slower as
+// well: 866 vs 1000 at GQA N=4096 d=128, since S then stays live in registers
+// for the whole pass.)
 constexpr int EXP2_POLY_PAIRS_OF_8 = 0;
 
 template <int D, bool CAUSAL>

@@ -48,8 +48,10 @@ def load(build_if_missing=True):
     global _lib
     if _lib is not None:
         return _lib
-    path = _build.LIB
-    if build_if_missing:
+    # FA_LIBRARY_PATH selects another build of libfa.so (e.g. to compare two
+    # builds in one process tree); by default the in-tree build is used
+    path = os.environ.get("FA_LIBRARY_PATH") or _build.LIB
+    if build_if_missing and not os.environ.get("FA_LIBRARY_PATH"):
         path = _build.build()
     if not os.path.exists(path):
         raise RuntimeError("libfa.so not found at %s; run python -m exact_io_aware_67_b200.build"
