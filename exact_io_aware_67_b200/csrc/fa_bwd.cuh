@@ -262,10 +262,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint8_t* smem = L::SLACK ? align_1024(smem_raw) : smem_raw;
 
   // ---------------------------------------------------------------- work item
-  const int nkv_blocks = (p.N + 127) / 128;
-  const int j = (int)(blockIdx.x % nkv_blocks);           // kv tile (low j = most work)
-  const int hk = (int)((blockIdx.x / nkv_blocks) % p.Hkv);
-  const int b = (int)(blockIdx.x / ((unsigned)nkv_blocks * p.Hkv));
+  // Blocks are dispatched roughly in index order.  Causal: the K/V tile
+  // index is slowest, so the longest blocks (tile j has nq - j query tiles)
+  // start first and the short ones fill the tail -- at B=2, Hkv=8, N=4096
+  // this took the main kernel from 737 to 912 TFLOP/s on B200.  Without the
+  // mask every tile of a sequence has the same work, and the tiles of one
+  // (sequence, kv head) stay adjacent so that they share Q and dO in L2.
+  const unsigned nkv_blocks = (unsigned)(p.N + 127) / 128;
+  const unsigned bh = (unsigned)p.Hkv * p.B;
+  const unsigned u = CAUSAL ? (blockIdx.x % bh) : (blockIdx.x / nkv_blocks);
+  const int j = (int)(CAUSAL ? blockIdx.x / bh : blockIdx.x % nkv_blocks);
+  const int hk = (int)(u % p.Hkv);
+  const int b = (int)(u / p.Hkv);
   int seq_start = 0, len = p.N, bcoord = b;
   if (p.cu_seqlens != nullptr) {
     seq_start = p.cu_seqlens[b];
