@@ -38,6 +38,9 @@ def load_library(path):
                                                    ctypes.c_int, ctypes.c_double,
                                                    ctypes.c_int, ctypes.c_int, ip]
     lib.oracle_attention_fwd_streaming.restype = ctypes.c_int
+    lib.oracle_softmax_rows.argtypes = [dp, ctypes.c_long, ctypes.c_int, ctypes.c_double,
+                                        ctypes.c_int, dp, dp, ctypes.c_int]
+    lib.oracle_softmax_rows.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -202,3 +205,22 @@ def attention_fwd_streaming(q, k, v, scale, causal, tile, tile_order=None):
     if rc != 0:
         raise RuntimeError("oracle_attention_fwd_streaming failed: %d" % rc)
     return o, lse
+
+
+def softmax_rows(s, scale, causal, nthreads=0):
+    """Row softmax of score matrices s [..., n, n] (raw q.k products): the
+    middle step of standard attention.  Row i of each n x n matrix is query
+    i; the logits are scale * s, with j > i masked when causal.  Returns
+    (p, lse), p shaped like s, lse shaped like s[..., 0]."""
+    s = _f64(s)
+    n = s.shape[-1]
+    if s.ndim < 2 or s.shape[-2] != n:
+        raise ValueError("s must be [..., n, n]")
+    rows = s.size // n
+    p = np.zeros(s.shape, dtype=np.float64)
+    lse = np.zeros(s.shape[:-1], dtype=np.float64)
+    rc = _load().oracle_softmax_rows(_dptr(s), rows, n, float(scale), int(bool(causal)),
+                                     _dptr(p), _dptr(lse), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle_softmax_rows failed: %d" % rc)
+    return p, lse

@@ -29,6 +29,10 @@
  *     query head h uses key/value head floor(h / (Hq/Hkv))).
  *   LSE_i = m_i + ln(l_i), natural log, in the scaled-logit domain.
  *
+ * oracle_softmax_rows is the middle step of standard attention alone -- the
+ * row softmax of score rows given as input -- for checking the standard-
+ * attention comparator, which materialises S and P in device memory.
+ *
  * The streaming variant (oracle_attention_fwd_streaming) follows the online
  * softmax recurrence of "FlashAttention优化" section 3.2.1 (running max m and
  * sum l, l_i = e^(m_{i-1}-m_i) l_{i-1} + sum exp(x_j - m_i)) together with the
@@ -458,6 +462,44 @@ int oracle_attention_fwd_streaming(const double* q, const double* k, const doubl
     free(x);
     free(acc);
     return 0;
+}
+
+/* The softmax step of standard attention on given score rows
+   ("注意力机制基础" 2.1 step 3; 2.2.2: S is read back and P written):
+   s holds rows of n raw scores q_i . k_j, row r belonging to query
+   i = r mod n of its head; the logit is scale * s_rj, -inf for j > i when
+   causal; each row then takes the three passes of softmax_row_three_pass.
+   p gets P (same layout as s), lse the natural-log LSE of each row. */
+int oracle_softmax_rows(const double* s, long rows, int n, double scale, int causal,
+                        double* p, double* lse, int nthreads) {
+    if (rows < 0 || n < 1 || !(scale > 0.0)) return -1;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+#endif
+    {
+        double* x = (double*)malloc(sizeof(double) * (size_t)n);
+        if (!x) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = -2;
+        }
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
+        for (long r = 0; r < rows; ++r) {
+            if (!x) continue;
+            const long i = r % n;
+            const double* srow = s + (size_t)r * n;
+            for (int j = 0; j < n; ++j)
+                x[j] = (causal && j > i) ? -INFINITY : scale * srow[j];
+            lse[r] = softmax_row_three_pass(x, n, p + (size_t)r * n);
+        }
+        free(x);
+    }
+    return err;
 }
 
 int oracle_num_threads(void) {

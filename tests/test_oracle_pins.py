@@ -279,3 +279,60 @@ def test_matches_torch_sdpa_fp64(N, Hq, Hkv, causal):
     np.testing.assert_allclose(g["dq"], dq_t, atol=1e-11)
     np.testing.assert_allclose(g["dk"], dk_t, atol=1e-11)
     np.testing.assert_allclose(g["dv"], dv_t, atol=1e-11)
+
+
+# ------------------------------------------------- softmax step of standard attention
+
+@pytest.mark.parametrize("n,causal", [(1, False), (5, True), (7, False), (16, True)])
+def test_softmax_rows_matches_brute_force(n, causal):
+    rng = np.random.default_rng(100 + n)
+    s = rng.standard_normal((3, n, n)) * 4.0
+    scale = 0.3
+    p, lse = oracle.softmax_rows(s, scale, causal)
+    for h in range(3):
+        for i in range(n):
+            row = [-math.inf if (causal and j > i) else scale * float(s[h, i, j])
+                   for j in range(n)]
+            bp, bl = brute._softmax(row)
+            np.testing.assert_allclose(p[h, i], bp, rtol=0, atol=1e-15)
+            assert abs(lse[h, i] - bl) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_softmax_rows_constant_rows(causal):
+    # every allowed logit equal: P uniform over the allowed keys and
+    # LSE = scale * c + ln(count)
+    n, c, scale = 9, 2.5, 0.7
+    p, lse = oracle.softmax_rows(np.full((2, n, n), c), scale, causal)
+    for i in range(n):
+        cnt = i + 1 if causal else n
+        np.testing.assert_allclose(p[:, i, :cnt], 1.0 / cnt, atol=1e-15)
+        assert np.all(p[:, i, cnt:] == 0.0)
+        np.testing.assert_allclose(lse[:, i], scale * c + math.log(cnt), atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_softmax_rows_matches_torch_softmax(causal):
+    rng = np.random.default_rng(7)
+    n, scale = 33, 0.125
+    s = rng.standard_normal((4, n, n)) * 8.0
+    x = torch.tensor(s, dtype=torch.float64) * scale
+    if causal:
+        x = x.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    p, lse = oracle.softmax_rows(s, scale, causal)
+    np.testing.assert_allclose(p, torch.softmax(x, dim=-1).numpy(), atol=1e-15)
+    np.testing.assert_allclose(lse, torch.logsumexp(x, dim=-1).numpy(), atol=1e-13)
+
+
+def test_standard_pipeline_equals_attention():
+    # S materialised, softmax step, then P V: the same O and LSE as the
+    # attention definition (one head per [n, n] matrix)
+    rng = np.random.default_rng(11)
+    N, H, d, scale = 40, 3, 8, 0.35
+    q, k, v = (rng.standard_normal((1, N, H, d)) for _ in range(3))
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, scale, True)
+    s = np.einsum("nhc,mhc->hnm", q[0], k[0])
+    p, lse = oracle.softmax_rows(s, scale, True)
+    o = np.einsum("hnm,mhc->nhc", p, v[0])
+    np.testing.assert_allclose(o, o_ref[0], atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref[0], atol=1e-13)
