@@ -13,6 +13,7 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "std_softmax.cuh"
 
 namespace {
 
@@ -286,6 +287,29 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (scratch == nullptr) return FA_ERR_CUDA;
   return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Hq, Hkv,
                 N, d, scale, causal, cu_seqlens, total_tokens, stream);
+}
+
+fa_status fa_std_softmax(const void* s, void* p, float* lse, int BH, int N, float scale,
+                         int causal, cudaStream_t stream) {
+  if (BH < 0 || N < 1) return FA_ERR_INVALID_ARG;
+  if (N % 8 != 0 || N > fa::STD_MAX_N) return FA_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if ((long long)BH * N > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (BH == 0) return FA_OK;
+  if (!s || !p || !lse || !aligned16(s) || !aligned16(p) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  const fa_status st = bind_device_of(s);
+  if (st != FA_OK) return st;
+  fa::StdSoftmaxParams prm{};
+  prm.s = static_cast<const __nv_bfloat16*>(s);
+  prm.p = static_cast<__nv_bfloat16*>(p);
+  prm.lse = lse;
+  prm.rows = (long)BH * N;
+  prm.n = N;
+  prm.causal = causal != 0;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = fa::launch_std_softmax(prm, stream);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "standard softmax launch");
 }
 
 int fa_device_error(void) {

@@ -24,7 +24,7 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
             "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events",
-            "fa_bwd_noalloc"]
+            "fa_bwd_noalloc", "fa_std_softmax"]
 
 # capacity of the fixed scratch behind fa_bwd_noalloc (include/fa.h)
 FA_BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -65,6 +65,8 @@ def load(build_if_missing=True):
     lib.fa_bwd.restype = c_int
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd_noalloc.restype = c_int
+    lib.fa_std_softmax.argtypes = [vp, vp, vp, c_int, c_int, c_float, c_int, vp]
+    lib.fa_std_softmax.restype = c_int
     lib.fa_bwd_workspace_size.argtypes = [c_int] * 5
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_device_error.argtypes = []
@@ -106,6 +108,12 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, cau
     the library or by this binding); see include/fa.h for its limits."""
     return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
                                  int(causal), cu_seqlens, total_tokens, stream)
+
+
+def fa_std_softmax(s, p, lse, BH, N, scale, causal, stream):
+    """Softmax step of standard attention over a materialised S (comparator
+    only); see include/fa.h."""
+    return load().fa_std_softmax(s, p, lse, BH, N, scale, int(causal), stream)
 
 
 def fa_bwd_workspace_size(B, Hq, N, d, total_tokens):
@@ -247,3 +255,30 @@ class Attention(torch.autograd.Function):
 def attention(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None):
     return Attention.apply(q, k, v, scale if scale is not None else q.shape[-1] ** -0.5,
                            causal, cu_seqlens, max_seqlen)
+
+
+# ------------------------------------------------------------ comparator
+
+def standard_attention_fwd(q, k, v, scale=None, causal=False):
+    """Standard attention with S and P materialised in device memory, for
+    comparison with fa_fwd ("注意力机制基础" 2.1 and 2.2.2): S = Q K^T and
+    O = P V are library GEMMs (cuBLAS through torch.matmul, bf16 in, bf16
+    out), and the row softmax between them is fa_std_softmax.  Inputs are
+    head-major [B, H, N, d] bf16 with the same number of heads (the layout
+    of the pages' per-head matrices); returns O [B, H, N, d] and LSE
+    [B, H, N].  Device memory: two B*H*N*N bf16 matrices."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, nm)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same [B, H, N, d] shape")
+    if scale is None:
+        scale = d ** -0.5
+    s = torch.matmul(q, k.transpose(-1, -2))            # [B, H, N, N]
+    p = torch.empty_like(s)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = fa_std_softmax(_ptr(s), _ptr(p), _ptr(lse), B * H, N, float(scale), causal, _stream())
+    if st != FA_OK:
+        raise FAError("fa_std_softmax", st)
+    del s
+    return torch.matmul(p, v), lse

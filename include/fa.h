@@ -139,6 +139,24 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
 /*
+ * Comparator only -- the softmax step of *standard* attention, which writes
+ * the N x N probability matrix that fa_fwd never forms ("注意力机制基础"
+ * 2.1 steps 2-3 and 2.2.2: S is read from and P written to device memory).
+ * With S = Q K^T computed by a library GEMM per head, this reads
+ *   s   : bf16 [BH][N][N], row i of head h at (h N + i) N (unscaled Q K^T)
+ * and writes
+ *   p   : bf16 [BH][N][N], P_ij = exp(scale S_ij - LSE_i) for allowed j, 0
+ *         for j > i when causal
+ *   lse : fp32 [BH][N], ln sum_j exp(scale S_ij) over the allowed j
+ * so that O = P V is a second library GEMM.  One pass over HBM: 2 bytes
+ * read and 2 written per element.  N must be a multiple of 8 and at most
+ * 32768 (FA_ERR_UNSUPPORTED otherwise); BH * N must fit in an int; s and p
+ * must not overlap.  Same pointer, device and error rules as fa_fwd.
+ */
+fa_status fa_std_softmax(const void* s, void* p, float* lse, int BH, int N, float scale,
+                         int causal, cudaStream_t stream);
+
+/*
  * Device-side error word shared by all kernels of the library: 0 when no
  * wait has timed out since the last fa_clear_device_error().  Reads device
  * memory synchronously on the current device; call after synchronising.

@@ -83,3 +83,16 @@ def test_build_command_targets_sm100a():
     cmd = build.nvcc_command("x.so")
     assert "arch=compute_100a,code=sm_100a" in cmd
     assert "-lineinfo" in cmd
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(N=12), 2), (dict(N=32776), 2), (dict(BH=-1), 1), (dict(N=0), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("inf")), 1), (dict(s=None), 1),
+    (dict(p=ctypes.c_void_p(4104)), 1), (dict(BH=1 << 20, N=4096), 1), (dict(BH=0), 0),
+])
+def test_std_softmax_rejects_bad_arguments(lib, kw, expect):
+    a = dict(s=ctypes.c_void_p(4096), p=ctypes.c_void_p(8192), lse=ctypes.c_void_p(12288), BH=2,
+             N=64, scale=0.125, causal=1)
+    a.update(kw)
+    assert ops.fa_std_softmax(a["s"], a["p"], a["lse"], a["BH"], a["N"], a["scale"],
+                              a["causal"], None) == expect
