@@ -8,6 +8,12 @@ One step = fa_fwd (O, LSE) + fa_bwd (dQ, dK, dV) over one batch of the
 workload, all through the C ABI of libfa.so.  FLOPs: forward 4 B H N^2 d
 (halved for causal), backward 2.5x forward.  Prints ONE JSON line (rank 0).
 
+A decode workload (``--workload decode_*``) times one decode step over a
+KV cache instead (fa_decode: split-KV attention of one new token per
+sequence); it is bound by HBM bandwidth, so that line reports GB/s of the
+algorithmic bytes (the valid K and V cache rows, q, o, lse) against the
+measured copy bandwidth.
+
 Multi-GPU (torchrun, one process per GPU): the path partitions into
 independent (sequence, kv-head group) problems, so each rank runs its own
 batch of the same shape (weak scaling) with no data-path collective; the
@@ -29,6 +35,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = ("attention fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak")
+DECODE_METRIC = "decode attention over a KV cache: GB/s of K/V cache read (bf16, 1×B200)"
+L2_FLUSH_BYTES = 256 << 20
 DEFAULT_WORKLOAD = "gqa_causal_b2_hq32_hkv8_n4096_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -390,6 +398,197 @@ def source_sha():
     return h.hexdigest()[:16]
 
 
+# ------------------------------------------------------------------ decode
+def decode_bytes(w, lengths):
+    """Algorithmic bytes of one decode step: every valid K and V cache row
+    read once, q read, o written (bf16) and lse written (fp32)."""
+    kv = sum(lengths) * w.Hkv * w.d * 2 * 2
+    return kv + w.B * w.Hq * w.d * 2 * 2 + w.B * w.Hq * 4
+
+
+def decode_cpu_sample(w, inp, nthreads, seqs=1):
+    """The oracle on `seqs` sequences of the decode step (every query head):
+    returns (seconds, algorithmic bytes of that sample)."""
+    import numpy as np
+    import oracle
+    lens = inp.lengths
+    t0 = time.perf_counter()
+    nbytes = 0
+    for b in range(seqs):
+        L = lens[b]
+        qf = np.zeros((1, L, w.Hq, w.d))
+        qf[0, 0] = inp.q[b].double().numpy()
+        rows = np.array([[0, h, 0] for h in range(w.Hq)])
+        oracle.attention_rows(qf, inp.k[b:b + 1, :L].double().numpy(),
+                              inp.v[b:b + 1, :L].double().numpy(), None, rows, w.scale, False,
+                              nthreads=nthreads)
+        nbytes += L * w.Hkv * w.d * 4 + w.Hq * w.d * 4 + w.Hq * 4
+    return time.perf_counter() - t0, nbytes
+
+
+def run_decode(args, w, impl):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_67_b200 import ops, workloads
+
+    ws, rank, local = dist_env()
+    cores = len(os.sched_getaffinity(0))
+    if impl == "reference":
+        if rank != 0:
+            return 0
+        inp = workloads.generate_decode(w)
+        for _ in range(args.warmup):
+            decode_cpu_sample(w, inp, cores)
+        tot_t, tot_b = 0.0, 0
+        for _ in range(args.steps):
+            dt, nb = decode_cpu_sample(w, inp, cores)
+            tot_t += dt
+            tot_b += nb
+        value = tot_b / tot_t / 1e9
+        sample = "1 sequence (all %d query heads, %d cached keys) of %s per step, fp64 oracle" % (
+            w.Hq, inp.lengths[0], w.name)
+        print(json.dumps({
+            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, **w.describe()},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    wr = workloads.DecodeWorkload(**{**w.__dict__, "seed": w.seed + rank})
+    inp = workloads.generate_decode(wr)
+    lengths = inp.lengths
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    sl = None if inp.seqlens is None else inp.seqlens.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    wsb = torch.empty(ops.fa_decode_workspace_size(w.B, w.Hq, w.Lmax, w.d), dtype=torch.uint8,
+                      device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    step_bytes = decode_bytes(w, lengths)
+    # a cache of more than twice the L2 (126 MB) evicts itself between steps;
+    # a smaller one is flushed by writing a buffer larger than the L2
+    flush_l2 = step_bytes < 2 * 126e6
+
+    def step():
+        ops.decode(q, k, v, sl, w.scale, out=o, lse=lse, workspace=wsb)
+
+    ops.fa_clear_device_error()
+    for _ in range(args.warmup):
+        if flush_l2:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        if flush_l2:
+            flush.zero_()                  # L2 flushed between timed steps
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    err = ops.fa_device_error()
+    if err != 0:
+        raise RuntimeError("device error word 0x%x during the timed region" % err)
+
+    # e2e: the new token's q, k and v from pinned host memory (k and v written
+    # into the cache at each sequence's last position), o and lse back
+    e2e = None
+    if not args.no_e2e:
+        hq = inp.q.pin_memory()
+        last = [max(L - 1, 0) for L in lengths]
+        hk = torch.stack([inp.k[b, last[b]] for b in range(w.B)]).pin_memory()
+        hv = torch.stack([inp.v[b, last[b]] for b in range(w.B)]).pin_memory()
+        dk, dv = torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev)
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        bidx = torch.arange(w.B, device=dev)
+        lidx = torch.tensor(last, device=dev)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        n_e2e = min(args.steps, 200)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        for it in range(1 + n_e2e):
+            if it == 1:
+                torch.cuda.synchronize()
+                e0.record(stream)
+            q.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            k[bidx, lidx] = dk
+            v[bidx, lidx] = dv
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e = {"ms": e0.elapsed_time(e1) * args.steps / n_e2e, "h2d": h2d, "d2h": d2h}
+
+    ms_max, e2e_max = max_over_ranks([ms, e2e["ms"] if e2e else 0.0], device=dev)
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks, peaks_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    value = ws * step_bytes * args.steps / (ms_max / 1e3) / 1e9
+    avg_ms = ms / args.steps
+    achieved = step_bytes / (avg_ms / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q and cache of the workload's shape)",
+        "config": {"workload": w.name, **w.describe(),
+                   "l2": ("flushed between timed steps (256 MB write)" if flush_l2 else
+                          "cache larger than twice the L2 (%.0f MB per step)" % (step_bytes / 1e6)),
+                   "parallelism": "independent batches per GPU" if ws > 1 else "1 GPU"},
+        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + decode_merge_kernel",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "algorithmic_bytes_per_launch": step_bytes, "avg_launch_ms": avg_ms,
+                     "peak_source": "%s hbm_gbs" % peaks_src},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if e2e:
+        line["e2e"] = {"value": ws * step_bytes * args.steps / (e2e_max / 1e3) / 1e9,
+                       "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                       "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e_max / args.steps}
+    if not args.no_cpu_baseline and ws == 1:
+        dt, nb = decode_cpu_sample(w, inp, cores)
+        line["cpu_baseline"] = {
+            "value": nb / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "seconds": dt,
+            "sample": "1 sequence (all %d query heads, %d cached keys), fp64 oracle" % (
+                w.Hq, lengths[0])}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,6 +600,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     from exact_io_aware_67_b200 import workloads
+    if args.workload in workloads.DECODE_WORKLOADS:
+        return run_decode(args, workloads.DECODE_WORKLOADS[args.workload], args.impl)
     w = workloads.WORKLOADS[args.workload]
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -12,6 +12,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 #include "std_softmax.cuh"
 
@@ -287,6 +288,66 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (scratch == nullptr) return FA_ERR_CUDA;
   return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Hq, Hkv,
                 N, d, scale, causal, cu_seqlens, total_tokens, stream);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d) {
+  if (B < 0 || Hq < 1 || Lmax < 1 || Lmax > (1 << 24) || (d != 64 && d != 128)) return 0;
+  return fa::decode_workspace_bytes(B, Hq, Lmax, d);
+}
+
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                    float* lse, const int* cache_seqlens, int B, int Hq, int Hkv, int Lmax,
+                    int d, float scale, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream) {
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (Hq / Hkv > fa::DEC_GMAX) return FA_ERR_UNSUPPORTED;
+  if (Lmax < 1 || Lmax > (1 << 24) || B > 65535 || Hkv > 65535) return FA_ERR_INVALID_ARG;
+  if ((long long)B * Hq > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k_cache, v_cache, o, lse};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if (cache_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  const size_t need = fa::decode_workspace_bytes(B, Hq, Lmax, d);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_WORKSPACE;
+  fa_status st = bind_device_of(q);
+  if (st != FA_OK) return st;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device attribute");
+
+  CUtensorMap mk, mv;
+  if (!encode_rows_map(&mk, k_cache, d, Hkv, Lmax, B) ||
+      !encode_rows_map(&mv, v_cache, d, Hkv, Lmax, B))
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
+  fa::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.seqlens = cache_seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lmax = Lmax;
+  p.group = Hq / Hkv;
+  fa::decode_plan(B, Hkv, Lmax, sms, &p.chunk, &p.splits);
+  if ((long long)B * Hkv * p.splits > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  p.items = B * Hkv * p.splits;
+  const size_t o_bytes = (size_t)p.splits * B * Hq * d * 4;
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        ((o_bytes + 255) & ~(size_t)255));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  e = fa::launch_decode(mk, mv, p, d, stream);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "decode launch");
 }
 
 fa_status fa_std_softmax(const void* s, void* p, float* lse, int BH, int N, float scale,

@@ -9,7 +9,7 @@
 namespace fa {
 
 // Codes written to the device error word when a bounded wait gives up:
-// 0x1xx forward kernel, 0x2xx backward kernels, 0x3xx self-test.
+// 0x1xx forward kernel, 0x2xx backward kernels, 0x3xx self-test, 0x4xx decode.
 enum : int {
   ERR_FWD_KV_EMPTY = 0x101,
   ERR_FWD_Q_FULL = 0x102,
@@ -32,6 +32,8 @@ enum : int {
   ERR_BWD_STATS = 0x20b,
   ERR_BWD_SMEM_ALIGN = 0x20c,
   ERR_SELFTEST = 0x301,
+  ERR_DEC_KV_FULL = 0x401,
+  ERR_DEC_KV_EMPTY = 0x402,
 };
 
 struct FwdParams {

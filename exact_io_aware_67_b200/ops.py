@@ -24,7 +24,7 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
             "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events",
-            "fa_bwd_noalloc", "fa_std_softmax"]
+            "fa_bwd_noalloc", "fa_std_softmax", "fa_decode", "fa_decode_workspace_size"]
 
 # capacity of the fixed scratch behind fa_bwd_noalloc (include/fa.h)
 FA_BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -65,6 +65,10 @@ def load(build_if_missing=True):
     lib.fa_bwd.restype = c_int
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd_noalloc.restype = c_int
+    lib.fa_decode.argtypes = [vp] * 6 + [c_int] * 5 + [c_float, vp, ctypes.c_size_t, vp]
+    lib.fa_decode.restype = c_int
+    lib.fa_decode_workspace_size.argtypes = [c_int] * 4
+    lib.fa_decode_workspace_size.restype = ctypes.c_size_t
     lib.fa_std_softmax.argtypes = [vp, vp, vp, c_int, c_int, c_float, c_int, vp]
     lib.fa_std_softmax.restype = c_int
     lib.fa_bwd_workspace_size.argtypes = [c_int] * 5
@@ -108,6 +112,16 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, cau
     the library or by this binding); see include/fa.h for its limits."""
     return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
                                  int(causal), cu_seqlens, total_tokens, stream)
+
+
+def fa_decode(q, k_cache, v_cache, o, lse, cache_seqlens, B, Hq, Hkv, Lmax, d, scale, workspace,
+              workspace_bytes, stream):
+    return load().fa_decode(q, k_cache, v_cache, o, lse, cache_seqlens, B, Hq, Hkv, Lmax, d,
+                            scale, workspace, workspace_bytes, stream)
+
+
+def fa_decode_workspace_size(B, Hq, Lmax, d):
+    return load().fa_decode_workspace_size(B, Hq, Lmax, d)
 
 
 def fa_std_softmax(s, p, lse, BH, N, scale, causal, stream):
@@ -255,6 +269,36 @@ class Attention(torch.autograd.Function):
 def attention(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None):
     return Attention.apply(q, k, v, scale if scale is not None else q.shape[-1] ** -0.5,
                            causal, cu_seqlens, max_seqlen)
+
+
+# ------------------------------------------------------------ decode
+
+def decode(q, k_cache, v_cache, cache_seqlens=None, scale=None, out=None, lse=None,
+           workspace=None):
+    """One decode step over a KV cache (fa_decode): q [B, Hq, d], caches
+    [B, Lmax, Hkv, d], cache_seqlens int32 [B] on the device or None (every
+    cache full).  Returns o [B, Hq, d] and lse [B, Hq]."""
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, nm)
+    B, Hq, d = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    if v_cache.shape != k_cache.shape or k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError("cache shapes must be [B, Lmax, Hkv, d] and match q")
+    if cache_seqlens is not None:
+        _check(cache_seqlens, "cache_seqlens", torch.int32)
+    if scale is None:
+        scale = d ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(fa_decode_workspace_size(B, Hq, Lmax, d), dtype=torch.uint8,
+                                device=q.device)
+    st = fa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                   _ptr(cache_seqlens), B, Hq, Hkv, Lmax, d, float(scale), _ptr(workspace),
+                   workspace.numel(), _stream())
+    if st != FA_OK:
+        raise FAError("fa_decode", st)
+    return out, lse
 
 
 # ------------------------------------------------------------ comparator

@@ -148,3 +148,79 @@ def from_lengths(name, lengths, Hq, Hkv, d, causal, seed=0):
     bf = torch.bfloat16
     return Inputs(q=q.to(bf), k=k.to(bf), v=v.to(bf), dout=dout.to(bf), cu_seqlens=cu,
                   workload=w, lengths=list(lengths))
+
+
+# ------------------------------------------------------------ decode over a KV cache
+
+@dataclass
+class DecodeWorkload:
+    """One decode step: B sequences, each with one new query token and a
+    cache of L_b keys and values (L_b = Lmax, or drawn uniformly in
+    ``lengths`` = (lo, hi) inclusive)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Lmax: int
+    d: int
+    scale: float
+    lengths: Optional[tuple] = None
+    seed: int = 0
+
+    def describe(self):
+        out = dict(B=self.B, Hq=self.Hq, Hkv=self.Hkv, Lmax=self.Lmax, d=self.d,
+                   scale=self.scale)
+        if self.lengths:
+            out["cache_lengths"] = list(self.lengths)
+        return out
+
+
+def _dw(name, B, Hq, Hkv, Lmax, d, lengths=None, seed=0):
+    return DecodeWorkload(name=name, B=B, Hq=Hq, Hkv=Hkv, Lmax=Lmax, d=d,
+                          scale=1.0 / math.sqrt(d), lengths=lengths, seed=seed)
+
+
+DECODE_WORKLOADS = {
+    # the tutorial's inference case study: batch 4, 8 heads of d = 64, a
+    # 2048-token prompt plus 512 generated tokens in the cache
+    "decode_b4_h8_l2560_d64": _dw("decode_b4_h8_l2560_d64", 4, 8, 8, 2560, 64),
+    # grouped-query decode of a long context, the shape of the GQA config
+    "decode_gqa_b8_hq32_hkv8_l8192_d128": _dw("decode_gqa_b8_hq32_hkv8_l8192_d128",
+                                              8, 32, 8, 8192, 128),
+    # a serving batch of mixed cache lengths
+    "decode_gqa_b16_hq32_hkv8_l1024to16384_d128": _dw(
+        "decode_gqa_b16_hq32_hkv8_l1024to16384_d128", 16, 32, 8, 16384, 128,
+        lengths=(1024, 16384)),
+}
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor          # [B, Hq, d]
+    k: torch.Tensor          # [B, Lmax, Hkv, d]
+    v: torch.Tensor          # [B, Lmax, Hkv, d]
+    seqlens: Optional[torch.Tensor]   # int32 [B] or None (all Lmax)
+    workload: DecodeWorkload
+
+    @property
+    def lengths(self):
+        w = self.workload
+        return [w.Lmax] * w.B if self.seqlens is None else [int(x) for x in self.seqlens]
+
+
+def generate_decode(w: DecodeWorkload) -> DecodeInputs:
+    """Draw a decode step's inputs on the CPU: cache lengths (if drawn), then
+    q, then the K cache, then the V cache, i.i.d. N(0, 1) rounded to bf16.
+    Cache rows past a sequence's length are drawn like the rest (a real
+    cache holds stale values there); the kernels must not use them."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    seqlens = None
+    if w.lengths:
+        lo, hi = w.lengths
+        seqlens = torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    q = torch.randn((w.B, w.Hq, w.d), generator=g, dtype=torch.float32)
+    k = torch.randn((w.B, w.Lmax, w.Hkv, w.d), generator=g, dtype=torch.float32)
+    v = torch.randn((w.B, w.Lmax, w.Hkv, w.d), generator=g, dtype=torch.float32)
+    bf = torch.bfloat16
+    return DecodeInputs(q=q.to(bf), k=k.to(bf), v=v.to(bf), seqlens=seqlens, workload=w)

@@ -139,6 +139,37 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                          const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
 /*
+ * Decode attention over a KV cache: one new query token per sequence
+ * attends to the first L_b cached keys and values of its sequence
+ * ("注意力机制基础" 2.3.1: autoregressive decoding re-reads the whole cache
+ * for every token; "FlashAttention优化" 4.2).  For each sequence b and
+ * query head h (key/value head h / (Hq / Hkv)):
+ *     o[b][h]   = sum_j softmax_j(scale q[b][h] . k[b][j]) v[b][j],  j < L_b
+ *     lse[b][h] = ln sum_j exp(scale q[b][h] . k[b][j])
+ *   q, o             : bf16 [B][Hq][d]
+ *   k_cache, v_cache : bf16 [B][Lmax][Hkv][d] (the training layout with
+ *                      N = Lmax); rows at or past L_b are never used, so they
+ *                      may hold anything
+ *   lse              : fp32 [B][Hq]
+ *   cache_seqlens    : device int32[B] with L_b (clamped to [0, Lmax]), or
+ *                      NULL for L_b = Lmax.  A sequence with L_b = 0 gets
+ *                      o = 0 and lse = -inf.
+ *   workspace        : caller-owned device memory of at least
+ *                      fa_decode_workspace_size() bytes, 256-byte aligned,
+ *                      for the per-chunk partial results
+ * The cache is cut into chunks processed in parallel and merged exactly
+ * (lse = ln sum_s e^(lse_s), o = sum_s e^(lse_s - lse) o_s).  d must be 64
+ * or 128 and Hq / Hkv at most 16 (FA_ERR_UNSUPPORTED otherwise); B and Hkv
+ * at most 65535.  Same pointer, device, error and stream rules as fa_fwd.
+ */
+size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d);
+
+fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, void* o,
+                    float* lse, const int* cache_seqlens, int B, int Hq, int Hkv, int Lmax,
+                    int d, float scale, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/*
  * Comparator only -- the softmax step of *standard* attention, which writes
  * the N x N probability matrix that fa_fwd never forms ("注意力机制基础"
  * 2.1 steps 2-3 and 2.2.2: S is read from and P written to device memory).

@@ -96,3 +96,25 @@ def test_std_softmax_rejects_bad_arguments(lib, kw, expect):
     a.update(kw)
     assert ops.fa_std_softmax(a["s"], a["p"], a["lse"], a["BH"], a["N"], a["scale"],
                               a["causal"], None) == expect
+
+
+def test_decode_rejects_bad_arguments(lib):
+    # host-side checks need no device work; sizes as for a valid call
+    p = ctypes.c_void_p(4096)
+    need = ops.fa_decode_workspace_size(2, 8, 512, 64)
+    ws = ctypes.c_void_p(4096)
+    args = lambda **kw: dict(dict(q=p, k=p, v=p, o=p, lse=p, sl=None, B=2, Hq=8, Hkv=2, L=512,
+                                  d=64, scale=0.125, ws=ws, wsb=need), **kw)
+
+    def call(a):
+        return ops.fa_decode(a["q"], a["k"], a["v"], a["o"], a["lse"], a["sl"], a["B"], a["Hq"],
+                             a["Hkv"], a["L"], a["d"], a["scale"], a["ws"], a["wsb"], None)
+    assert call(args(d=96)) == 2
+    assert call(args(Hq=34, Hkv=2)) == 2          # 17 query heads per kv head
+    assert call(args(Hq=7)) == 1
+    assert call(args(L=0)) == 1
+    assert call(args(scale=0.0)) == 1
+    assert call(args(wsb=need - 1)) == 3
+    assert call(args(ws=ctypes.c_void_p(4096 + 16))) == 3
+    assert call(args(q=ctypes.c_void_p(4100))) == 1
+    assert call(args(B=0)) == 0
