@@ -38,6 +38,13 @@ def load_library(path):
                                                    ctypes.c_int, ctypes.c_double,
                                                    ctypes.c_int, ctypes.c_int, ip]
     lib.oracle_attention_fwd_streaming.restype = ctypes.c_int
+    bp = ctypes.POINTER(ctypes.c_ubyte)
+    maskc = [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int, bp, ctypes.c_long,
+                                  ctypes.c_long, ctypes.c_int]
+    lib.oracle_attention_fwd_blockmask.argtypes = [dp, dp, dp, dp, dp] + maskc
+    lib.oracle_attention_fwd_blockmask.restype = ctypes.c_int
+    lib.oracle_attention_bwd_blockmask.argtypes = [dp] * 10 + maskc
+    lib.oracle_attention_bwd_blockmask.restype = ctypes.c_int
     lib.oracle_softmax_rows.argtypes = [dp, ctypes.c_long, ctypes.c_int, ctypes.c_double,
                                         ctypes.c_int, dp, dp, ctypes.c_int]
     lib.oracle_softmax_rows.restype = ctypes.c_int
@@ -224,3 +231,59 @@ def softmax_rows(s, scale, causal, nthreads=0):
     if rc != 0:
         raise RuntimeError("oracle_softmax_rows failed: %d" % rc)
     return p, lse
+
+
+def _mask(block_mask):
+    """uint8 [Bm, Hm, nt, nt] with Bm in {1, B} and Hm in {1, Hkv}: returns
+    the array and its (sequence, head) strides in elements (0 broadcasts)."""
+    bm = np.ascontiguousarray(np.asarray(block_mask, dtype=np.uint8))
+    if bm.ndim != 4 or bm.shape[2] != bm.shape[3]:
+        raise ValueError("block mask must be [Bm, Hm, nt, nt]")
+    nt = bm.shape[2]
+    sb = 0 if bm.shape[0] == 1 else bm.shape[1] * nt * nt
+    sh = 0 if bm.shape[1] == 1 else nt * nt
+    return bm, sb, sh
+
+
+def attention_fwd_blockmask(q, k, v, scale, causal, block_mask, nthreads=0):
+    """O and LSE of block-sparse attention (dense layout): the definition with
+    every (query, key) pair whose 128 x 128 tile is not allowed by the block
+    mask of its key/value head removed.  block_mask: [Bm, Hm, nt, nt] with
+    nt = ceil(N / 128), Bm in {1, B}, Hm in {1, Hkv} (1 broadcasts)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    bm, sb, sh = _mask(block_mask)
+    if bm.shape[2] != (N + 127) // 128 or bm.shape[0] not in (1, B) or bm.shape[1] not in (1, Hkv):
+        raise ValueError("block mask shape %s does not fit B=%d Hkv=%d N=%d" % (bm.shape, B, Hkv, N))
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, Hq, N), dtype=np.float64)
+    rc = _load().oracle_attention_fwd_blockmask(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(o), _dptr(lse), B, Hq, Hkv, N, d, float(scale),
+        int(bool(causal)), bm.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)), sb, sh,
+        int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle_attention_fwd_blockmask failed: %d" % rc)
+    return o, lse
+
+
+def attention_bwd_blockmask(q, k, v, dout, scale, causal, block_mask, nthreads=0):
+    """dQ, dK, dV (plus O, LSE, D) of block-sparse attention; see
+    attention_fwd_blockmask."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    bm, sb, sh = _mask(block_mask)
+    if bm.shape[2] != (N + 127) // 128 or bm.shape[0] not in (1, B) or bm.shape[1] not in (1, Hkv):
+        raise ValueError("block mask shape %s does not fit B=%d Hkv=%d N=%d" % (bm.shape, B, Hkv, N))
+    dq, dk, dv = (np.zeros(t.shape, dtype=np.float64) for t in (q, k, v))
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, Hq, N), dtype=np.float64)
+    D = np.zeros_like(lse)
+    rc = _load().oracle_attention_bwd_blockmask(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(dout), _dptr(dq), _dptr(dk), _dptr(dv), _dptr(o),
+        _dptr(lse), _dptr(D), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+        bm.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)), sb, sh, int(nthreads))
+    if rc != 0:
+        raise RuntimeError("oracle_attention_bwd_blockmask failed: %d" % rc)
+    return {"dq": dq, "dk": dk, "dv": dv, "o": o, "lse": lse, "D": D}

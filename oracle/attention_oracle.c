@@ -62,11 +62,18 @@
 #endif
 
 #define ORACLE_ROW_BLOCK 64
+#define ORACLE_MASK_TILE 128   /* block-mask granularity: 128 x 128 (query, key) tiles */
 
 typedef struct {
     int B, Hq, Hkv, N, d, causal, g;
     double scale;
     const int* cu;
+    /* optional block mask (dense layout only): tile (ti, tj) of sequence b
+       and key/value head hk is allowed iff
+       bm[b * bm_sb + hk * bm_sh + ti * bm_nt + tj] != 0 */
+    const unsigned char* bm;
+    long bm_sb, bm_sh;
+    int bm_nt;
 } shape_t;
 
 /* number of sequences and the token range of sequence s */
@@ -120,6 +127,14 @@ static void score_row(const shape_t* sh, const double* q, const double* k,
             srow[j] = -INFINITY;
             continue;
         }
+        if (sh->bm) {
+            const long b = start / sh->N;
+            if (!sh->bm[b * sh->bm_sb + hk * sh->bm_sh + (long)(i / ORACLE_MASK_TILE) * sh->bm_nt +
+                        j / ORACLE_MASK_TILE]) {
+                srow[j] = -INFINITY;
+                continue;
+            }
+        }
         const double* kj = k + tok_off(sh, start + j, hk, sh->Hkv);
         double acc = 0.0;
         for (int c = 0; c < d; ++c) acc += qi[c] * kj[c];
@@ -133,6 +148,12 @@ static double softmax_row_three_pass(const double* srow, int len, double* prow) 
     double m = -INFINITY;
     for (int j = 0; j < len; ++j)
         if (srow[j] > m) m = srow[j];
+    if (m == -INFINITY) {
+        /* no allowed key (a block mask can remove them all): P = 0, and the
+           log of the empty sum is -inf */
+        for (int j = 0; j < len; ++j) prow[j] = 0.0;
+        return -INFINITY;
+    }
     double l = 0.0;
     for (int j = 0; j < len; ++j) {
         double e = (srow[j] == -INFINITY) ? 0.0 : exp(srow[j] - m);
@@ -145,11 +166,9 @@ static double softmax_row_three_pass(const double* srow, int len, double* prow) 
 
 static int nseq(const shape_t* sh) { return sh->B; }
 
-int oracle_attention_fwd(const double* q, const double* k, const double* v,
-                         double* o, double* lse,
-                         int B, int Hq, int Hkv, int N, int d, double scale,
-                         int causal, const int* cu_seqlens, int nthreads) {
-    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens};
+static int attention_fwd_sh(shape_t sh, const double* q, const double* k, const double* v,
+                            double* o, double* lse, int nthreads) {
+    const int Hq = sh.Hq, Hkv = sh.Hkv, d = sh.d;
     if (check_args(&sh)) return -1;
     sh.g = Hq / Hkv;
     int maxlen = 0;
@@ -213,13 +232,11 @@ int oracle_attention_fwd(const double* q, const double* k, const double* v,
     return err;
 }
 
-int oracle_attention_bwd(const double* q, const double* k, const double* v,
-                         const double* dout,
-                         double* dq, double* dk, double* dv,
-                         double* o, double* lse, double* Dout,
-                         int B, int Hq, int Hkv, int N, int d, double scale,
-                         int causal, const int* cu_seqlens, int nthreads) {
-    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens};
+static int attention_bwd_sh(shape_t sh, const double* q, const double* k, const double* v,
+                            const double* dout, double* dq, double* dk, double* dv,
+                            double* o, double* lse, double* Dout, int nthreads) {
+    const int Hq = sh.Hq, Hkv = sh.Hkv, d = sh.d;
+    const double scale = sh.scale;
     if (check_args(&sh)) return -1;
     sh.g = Hq / Hkv;
     int maxlen = 0;
@@ -320,6 +337,56 @@ int oracle_attention_bwd(const double* q, const double* k, const double* v,
     return err;
 }
 
+int oracle_attention_fwd(const double* q, const double* k, const double* v,
+                         double* o, double* lse,
+                         int B, int Hq, int Hkv, int N, int d, double scale,
+                         int causal, const int* cu_seqlens, int nthreads) {
+    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens, NULL, 0, 0, 0};
+    return attention_fwd_sh(sh, q, k, v, o, lse, nthreads);
+}
+
+int oracle_attention_bwd(const double* q, const double* k, const double* v,
+                         const double* dout,
+                         double* dq, double* dk, double* dv,
+                         double* o, double* lse, double* Dout,
+                         int B, int Hq, int Hkv, int N, int d, double scale,
+                         int causal, const int* cu_seqlens, int nthreads) {
+    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens, NULL, 0, 0, 0};
+    return attention_bwd_sh(sh, q, k, v, dout, dq, dk, dv, o, lse, Dout, nthreads);
+}
+
+/* Block-sparse attention (dense layout only): the same definition with S_ij
+   also set to -inf when the 128 x 128 tile that holds (i, j) is not allowed
+   by the block mask of the key/value head (a generalisation of the causal
+   tile skipping, "FlashAttention优化" 7.2 and the paper review's block-
+   sparse variant; exact on the allowed entries).  bm is
+   [*][*][ceil(N/128)][ceil(N/128)] bytes with strides bm_sb per sequence
+   and bm_sh per key/value head (0 broadcasts).  A row with no allowed key
+   gets P = 0, O = 0 and LSE = -inf. */
+int oracle_attention_fwd_blockmask(const double* q, const double* k, const double* v,
+                                   double* o, double* lse,
+                                   int B, int Hq, int Hkv, int N, int d, double scale,
+                                   int causal, const unsigned char* bm, long bm_sb,
+                                   long bm_sh, int nthreads) {
+    if (!bm) return -1;
+    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, NULL, bm, bm_sb, bm_sh,
+                  (N + ORACLE_MASK_TILE - 1) / ORACLE_MASK_TILE};
+    return attention_fwd_sh(sh, q, k, v, o, lse, nthreads);
+}
+
+int oracle_attention_bwd_blockmask(const double* q, const double* k, const double* v,
+                                   const double* dout,
+                                   double* dq, double* dk, double* dv,
+                                   double* o, double* lse, double* Dout,
+                                   int B, int Hq, int Hkv, int N, int d, double scale,
+                                   int causal, const unsigned char* bm, long bm_sb,
+                                   long bm_sh, int nthreads) {
+    if (!bm) return -1;
+    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, NULL, bm, bm_sb, bm_sh,
+                  (N + ORACLE_MASK_TILE - 1) / ORACLE_MASK_TILE};
+    return attention_bwd_sh(sh, q, k, v, dout, dq, dk, dv, o, lse, Dout, nthreads);
+}
+
 /* Query-row sample: O, LSE, D and dQ of the listed rows only.  Each row is
    computed from its own full S row, so the cost is O(len * d) per row.
    rows[3*r .. 3*r+2] = (sequence s, query head h, row i within sequence). */
@@ -329,7 +396,7 @@ int oracle_attention_rows(const double* q, const double* k, const double* v,
                           double* dq_rows,
                           int B, int Hq, int Hkv, int N, int d, double scale,
                           int causal, const int* cu_seqlens, int nthreads) {
-    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens};
+    shape_t sh = {B, Hq, Hkv, N, d, causal, 0, scale, cu_seqlens, NULL, 0, 0, 0};
     if (check_args(&sh)) return -1;
     sh.g = Hq / Hkv;
     for (long r = 0; r < nrows; ++r) {

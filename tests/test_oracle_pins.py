@@ -336,3 +336,131 @@ def test_standard_pipeline_equals_attention():
     o = np.einsum("hnm,mhc->nhc", p, v[0])
     np.testing.assert_allclose(o, o_ref[0], atol=1e-13)
     np.testing.assert_allclose(lse, lse_ref[0], atol=1e-13)
+
+
+# ------------------------------------------------------------------ block masks
+
+def _bm_problem(B=1, N=300, Hq=4, Hkv=2, d=8, seed=21):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    do = rng.standard_normal((B, N, Hq, d))
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blockmask_all_allowed_equals_unmasked(causal):
+    q, k, v, do = _bm_problem()
+    nt = 3
+    bm = np.ones((1, 1, nt, nt), dtype=np.uint8)
+    o, lse = oracle.attention_fwd_blockmask(q, k, v, 0.3, causal, bm)
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, 0.3, causal)
+    assert np.array_equal(o, o_ref) and np.array_equal(lse, lse_ref)
+    g = oracle.attention_bwd_blockmask(q, k, v, do, 0.3, causal, bm)
+    r = oracle.attention_bwd(q, k, v, do, 0.3, causal)
+    for nm in ("dq", "dk", "dv"):
+        assert np.array_equal(g[nm], r[nm])
+
+
+def test_blockmask_diagonal_equals_independent_sequences():
+    # only the diagonal 128 x 128 tiles allowed, non-causal: every 128-token
+    # block attends to itself alone, which is varlen attention over
+    # sequences of 128, 128, ..., the rest (a different indexing path)
+    q, k, v, do = _bm_problem(N=3 * 128 + 50)
+    N = q.shape[1]
+    nt = 4
+    bm = np.eye(nt, dtype=np.uint8)[None, None]
+    o, lse = oracle.attention_fwd_blockmask(q, k, v, 0.35, False, bm)
+    g = oracle.attention_bwd_blockmask(q, k, v, do, 0.35, False, bm)
+    cu = np.array([0, 128, 256, 384, N], dtype=np.int32)
+    o_v, lse_v = oracle.attention_fwd(q[0], k[0], v[0], 0.35, False, cu)
+    r = oracle.attention_bwd(q[0], k[0], v[0], do[0], 0.35, False, cu)
+    np.testing.assert_allclose(o[0], o_v, atol=1e-14)
+    np.testing.assert_allclose(lse[0], lse_v, atol=1e-14)
+    for nm in ("dq", "dk", "dv"):
+        np.testing.assert_allclose(g[nm][0], r[nm], atol=1e-13)
+
+
+def _sdpa_masked(q, k, v, do, scale, causal, bm):
+    """PyTorch fp64 SDPA with the block mask expanded to a boolean element
+    mask (per key/value head, repeated over its query heads)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    el = np.repeat(np.repeat(bm, 128, axis=2), 128, axis=3)[:, :, :N, :N].astype(bool)
+    el = np.broadcast_to(el, (B, Hkv, N, N))
+    if causal:
+        el = el & np.tril(np.ones((N, N), dtype=bool))
+    mask = torch.tensor(np.repeat(el, g, axis=1).copy())
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k, requires_grad=True)
+    tv = torch.tensor(v, requires_grad=True)
+    kk = tk.repeat_interleave(g, dim=2)
+    vv = tv.repeat_interleave(g, dim=2)
+    o = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(1, 2), kk.transpose(1, 2), vv.transpose(1, 2), attn_mask=mask,
+        scale=scale).transpose(1, 2)
+    return o, tq, tk, tv, mask
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blockmask_matches_torch_sdpa_with_element_mask(causal):
+    q, k, v, do = _bm_problem(B=2, N=300, Hq=4, Hkv=2, seed=5)
+    rng = np.random.default_rng(9)
+    bm = (rng.random((2, 2, 3, 3)) < 0.6).astype(np.uint8)
+    bm[:, :, np.arange(3), np.arange(3)] = 1          # every row keeps a key
+    o_t, tq, tk, tv, _ = _sdpa_masked(q, k, v, do, 0.3, causal, bm)
+    o_t.backward(torch.tensor(do))
+    o, _ = oracle.attention_fwd_blockmask(q, k, v, 0.3, causal, bm)
+    g = oracle.attention_bwd_blockmask(q, k, v, do, 0.3, causal, bm)
+    np.testing.assert_allclose(o, o_t.detach().numpy(), atol=1e-12)
+    np.testing.assert_allclose(g["dq"], tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(g["dk"], tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(g["dv"], tv.grad.numpy(), atol=1e-11)
+
+
+def test_blockmask_rows_without_keys():
+    # query tile 1 allowed nowhere: its rows get O = 0, LSE = -inf, dQ = 0
+    # and contribute nothing to dK, dV
+    q, k, v, do = _bm_problem(N=300)
+    bm = np.ones((1, 1, 3, 3), dtype=np.uint8)
+    bm[0, 0, 1, :] = 0
+    o, lse = oracle.attention_fwd_blockmask(q, k, v, 0.3, False, bm)
+    g = oracle.attention_bwd_blockmask(q, k, v, do, 0.3, False, bm)
+    assert np.all(o[:, 128:256] == 0.0) and np.all(np.isneginf(lse[:, :, 128:256]))
+    assert np.all(g["dq"][:, 128:256] == 0.0)
+    # the other rows are the unmasked problem with those query rows removed:
+    # zeroing dO on them leaves dK and dV of the full problem unchanged
+    do2 = do.copy()
+    do2[:, 128:256] = 0.0
+    r = oracle.attention_bwd(q, k, v, do2, 0.3, False)
+    np.testing.assert_allclose(g["dk"], r["dk"], atol=1e-12)
+    np.testing.assert_allclose(g["dv"], r["dv"], atol=1e-12)
+    np.testing.assert_allclose(o[:, :128], r["o"][:, :128], atol=1e-14)
+
+
+def test_blockmask_finite_differences():
+    q, k, v, do = _bm_problem(N=140, Hq=2, Hkv=1, d=4, seed=3)
+    bm = np.array([[[[1, 0], [1, 1]]]], dtype=np.uint8)
+    bm[0, 0, 1, 0] = 0                                 # row tile 1 sees only tile 1
+    scale, causal = 0.5, True
+    g = oracle.attention_bwd_blockmask(q, k, v, do, scale, causal, bm)
+
+    def loss():
+        o, _ = oracle.attention_fwd_blockmask(q, k, v, scale, causal, bm)
+        return float(np.sum(o * do))
+
+    h = 1e-6
+    for nm, arr, ixs in (("dq", q, [(0, 3, 1, 2), (0, 131, 0, 1)]),
+                         ("dk", k, [(0, 2, 0, 3), (0, 135, 0, 0)]),
+                         ("dv", v, [(0, 5, 0, 1), (0, 139, 0, 2)])):
+        for ix in ixs:
+            a0 = arr[ix]
+            arr[ix] = a0 + h
+            lp = loss()
+            arr[ix] = a0 - h
+            lm = loss()
+            arr[ix] = a0
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - g[nm][ix]) <= 1e-6 * max(1.0, abs(g[nm][ix])), (nm, ix, fd, g[nm][ix])
