@@ -120,10 +120,10 @@ fa_status check_dims(const Dims& s, float scale, bool* empty) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE = false>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const fa::FwdParams& p, cudaStream_t stream) {
-  auto kern = fa::fwd_kernel<D, CAUSAL>;
+  auto kern = fa::fwd_kernel<D, CAUSAL, SPARSE>;
   const int smem = fa::FwdLayout<D>::ALLOC;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -165,9 +165,28 @@ void* scratch_on_current_device() {
 
 extern "C" {
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                 int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
-                 int total_tokens, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Block mask of the block-sparse entry points: bytes [*][*][nt][nt] with
+// nt = ceil(N / 128), strides (in elements) per sequence and per kv head.
+struct BlockMask {
+  const unsigned char* m;
+  long sb, sh;
+};
+
+fa_status check_mask(const BlockMask& bm, const void* cu_seqlens, int N) {
+  if (bm.m == nullptr) return FA_OK;
+  if (cu_seqlens != nullptr) return FA_ERR_UNSUPPORTED;   // dense batches only
+  if ((N + 127) / 128 > fa::FA_SPARSE_MAX_TILES) return FA_ERR_UNSUPPORTED;
+  if (bm.sb < 0 || bm.sh < 0) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
+                   int total_tokens, const BlockMask& bm, cudaStream_t stream) {
   const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
   bool empty = false;
   fa_status st = check_dims(s, scale, &empty);
@@ -175,6 +194,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
+  st = check_mask(bm, cu_seqlens, N);
+  if (st != FA_OK) return st;
   if (empty) return FA_OK;
   st = bind_device_of(q);
   if (st != FA_OK) return st;
@@ -198,30 +219,37 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.num_qblocks = (N + 255) / 256;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.bmask = bm.m;
+  p.bm_sb = bm.sb;
+  p.bm_sh = bm.sh;
+  p.bm_nt = (N + 127) / 128;
 
   cudaError_t e;
-  if (d == 64)
-    e = causal ? launch_fwd<64, true>(mq, mk, mv, p, stream)
-               : launch_fwd<64, false>(mq, mk, mv, p, stream);
-  else
-    e = causal ? launch_fwd<128, true>(mq, mk, mv, p, stream)
-               : launch_fwd<128, false>(mq, mk, mv, p, stream);
+  if (bm.m == nullptr) {
+    if (d == 64)
+      e = causal ? launch_fwd<64, true>(mq, mk, mv, p, stream)
+                 : launch_fwd<64, false>(mq, mk, mv, p, stream);
+    else
+      e = causal ? launch_fwd<128, true>(mq, mk, mv, p, stream)
+                 : launch_fwd<128, false>(mq, mk, mv, p, stream);
+  } else {
+    if (d == 64)
+      e = causal ? launch_fwd<64, true, true>(mq, mk, mv, p, stream)
+                 : launch_fwd<64, false, true>(mq, mk, mv, p, stream);
+    else
+      e = causal ? launch_fwd<128, true, true>(mq, mk, mv, p, stream)
+                 : launch_fwd<128, false, true>(mq, mk, mv, p, stream);
+  }
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "forward launch");
 }
 
-size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
-  if (B < 0 || Hq < 1 || N < 1 || (d != 64 && d != 128) || total_tokens < 0) return 0;
-  // the size must serve a dense call (total_tokens = B * N) and a varlen
-  // call with the same numbers, so take the larger of the two layouts
-  const size_t a = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, false);
-  const size_t v = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, true);
-  return a > v ? a : v;
-}
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
-                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
-                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
+
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                   int causal, const int* cu_seqlens, int total_tokens, const BlockMask& bm,
+                   cudaStream_t stream) {
   const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
   bool empty = false;
   fa_status st = check_dims(s, scale, &empty);
@@ -230,6 +258,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  st = check_mask(bm, cu_seqlens, N);
+  if (st != FA_OK) return st;
   if (empty) return FA_OK;
   const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d, s.tokens(), s.varlen);
   if (workspace == nullptr || workspace_bytes < need ||
@@ -263,11 +293,63 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = g_wait_limit_ns.load();
+  p.bmask = bm.m;
+  p.bm_sb = bm.sb;
+  p.bm_sh = bm.sh;
+  p.bm_nt = (N + 127) / 128;
   fa::bwd_carve_workspace(p, workspace, s.tokens(), d);
 
   const cudaError_t e =
       fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream, t_prof_begin, t_prof_end);
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "backward launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
+                 int total_tokens, cudaStream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, total_tokens,
+                  BlockMask{nullptr, 0, 0}, stream);
+}
+
+fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int Hq, int Hkv, int N, int d, float scale, int causal,
+                           const unsigned char* block_mask, long mask_batch_stride,
+                           long mask_head_stride, cudaStream_t stream) {
+  if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, nullptr, B * N,
+                  BlockMask{block_mask, mask_batch_stride, mask_head_stride}, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
+  if (B < 0 || Hq < 1 || N < 1 || (d != 64 && d != 128) || total_tokens < 0) return 0;
+  // the size must serve a dense call (total_tokens = B * N) and a varlen
+  // call with the same numbers, so take the larger of the two layouts
+  const size_t a = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, false);
+  const size_t v = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, true);
+  return a > v ? a : v;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
+                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+                  scale, causal, cu_seqlens, total_tokens, BlockMask{nullptr, 0, 0}, stream);
+}
+
+fa_status fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                           void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
+                           int d, float scale, int causal, const unsigned char* block_mask,
+                           long mask_batch_stride, long mask_head_stride, cudaStream_t stream) {
+  if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+                  scale, causal, nullptr, B * N,
+                  BlockMask{block_mask, mask_batch_stride, mask_head_stride}, stream);
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,

@@ -65,6 +65,11 @@ struct BwdParams {
   int B, Hq, Hkv, N, group, total;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
+  // block-sparse mode only: tile (qt, kt) of sequence b and kv head hk is
+  // allowed iff bmask[b * bm_sb + hk * bm_sh + qt * bm_nt + kt] != 0
+  const uint8_t* bmask;
+  long bm_sb, bm_sh;
+  int bm_nt;
 };
 
 inline size_t bwd_dsum_bytes(int Hq, long tokens) {
@@ -224,7 +229,12 @@ struct BwdLayout {
   // p_full ds_full ds_empty dq_full dq_empty dkv_done drain
   static constexpr int NBAR = 20;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  // block-sparse mode: which query tiles the CTA's K/V tile meets (bits
+  // [FA_SPARSE_MAX_TILES / 32]) and how many
+  static constexpr int OFF_QBITS = OFF_MISC + 16;
+  static constexpr int OFF_NQ = OFF_QBITS + (FA_SPARSE_MAX_TILES / 32) * 4;
+  static constexpr int BYTES = OFF_NQ + 16;
+  static_assert(BYTES <= 232448, "shared memory per block");
   // The d = 128 layout uses all but ~0.8 KB of the 227 KB a CTA may have, so
   // it relies on the dynamic shared memory window starting 1024-byte aligned
   // (checked at run time; a misaligned base reports ERR_BWD_SMEM_ALIGN).
@@ -246,7 +256,17 @@ constexpr int BWD_REGS_DRAIN = 176;   // warpgroup 2 after setmaxnreg.inc
 constexpr int BWD_REGS_CTRL = 80;     // warpgroup 3 after setmaxnreg.dec
 static_assert(128 * (128 + 128 + BWD_REGS_DRAIN + BWD_REGS_CTRL) == 65536, "register split");
 
-template <int D, bool CAUSAL>
+// First set bit at or after position `from` of a bit list, or `limit`.
+__device__ __forceinline__ int next_set_bit(const uint32_t* bits, int from, int limit) {
+  for (int w = from >> 5; (w << 5) < limit; ++w) {
+    uint32_t x = bits[w];
+    if (w == (from >> 5)) x &= ~0u << (from & 31);
+    if (x != 0u) return min(limit, (w << 5) + __ffs(x) - 1);
+  }
+  return limit;
+}
+
+template <int D, bool CAUSAL, bool SPARSE = false>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -283,8 +303,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (128 * j >= len) return;
   const int nq = (len + 127) / 128;
   const int i0 = CAUSAL ? j : 0;
-  const int n_i = nq - i0;                  // query tiles per head
-  const int T = p.group * n_i;              // iterations of this CTA
+  // Block-sparse: the query tiles this K/V tile meets are those the block
+  // mask of its kv head allows (on or below the diagonal when causal); every
+  // query head of the group walks the same list, found once here.
+  uint32_t* s_qbits = reinterpret_cast<uint32_t*>(smem + L::OFF_QBITS);
+  int* s_nq = reinterpret_cast<int*>(smem + L::OFF_NQ);
+  if (SPARSE && warp == 14) {
+    const uint8_t* mcol = p.bmask + (long)b * p.bm_sb + (long)hk * p.bm_sh + j;
+    int cnt = 0;
+    for (int c0 = 0; c0 < FA_SPARSE_MAX_TILES; c0 += 32) {
+      const int i = c0 + lane;
+      const bool a = i >= i0 && i < nq && mcol[(long)i * p.bm_nt] != 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, a);
+      if (lane == 0) s_qbits[c0 >> 5] = bal;
+      cnt += __popc(bal);
+    }
+    if (lane == 0) *s_nq = cnt;
+  }
 
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
@@ -347,8 +382,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
+  const int n_i = SPARSE ? *s_nq : nq - i0;   // query tiles per head
+  const int T = p.group * n_i;                // iterations of this CTA
+  // query tile of iteration n (iterations run head by head over the list);
+  // `cur` carries the previous answer, so each role calls it with n = 0, 1, ...
+  auto qtile = [&](int n, int& cur) -> int {
+    if (!SPARSE) return i0 + n % n_i;
+    cur = next_set_bit(s_qbits, (n % n_i == 0) ? 0 : cur + 1, nq);
+    return cur;
+  };
 
-  if (warp >= 12) {
+  if (SPARSE && n_i == 0) {
+    // no query tile meets this K/V tile: dK = dV = 0 for its rows
+    for (int e = threadIdx.x; e < 128 * (D / 8); e += BWD_THREADS) {
+      const int r = e / (D / 8), c8 = e % (D / 8);
+      const int kv_row = 128 * j + r;
+      if (kv_row < len) {
+        const long t = (long)b * p.N + kv_row;
+        reinterpret_cast<uint4*>(p.dk + (t * p.Hkv + hk) * (long)D)[c8] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(p.dv + (t * p.Hkv + hk) * (long)D)[c8] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  } else if (warp >= 12) {
   // ============================================================== warpgroup 3
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(BWD_REGS_CTRL));
   if (warp == 12) {
@@ -364,9 +419,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     int q_issued = 0, do_issued = 0;
     bool ok = true;
+    int qcur = 0;
     for (int n = 0; n < T && ok; ++n) {
       const int h = hk * p.group + n / n_i;
-      const int i = i0 + n % n_i;
+      const int i = qtile(n, qcur);
       const int s = n & 1;
       const uint32_t ph_empty = ((n >> 1) & 1) ^ 1;
       // Q_n (stage s) and dO_n (stage s) by TMA
@@ -541,9 +597,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tq = tmem + lane_off + L::T_DQ;
     const long tb = tile_base(p, b);
+    int qcur = 0;
     for (int n = 0; n < T; ++n) {
       const int h = hk * p.group + n / n_i;
-      const int i = i0 + n % n_i;
+      const int i = qtile(n, qcur);
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, n & 1, wd, ERR_BWD_DQ_FULL))) break;
       tc_fence_after();
       uint32_t v[D];
@@ -578,8 +635,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // byte offset of this thread's row inside its 64-column dS region
     uint8_t* ds_row = sDS + wg * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
+    int qcur = 0;
     for (int n = 0; n < T; ++n) {
-      const int i = i0 + n % n_i;
+      const int i = qtile(n, qcur);
       const int s = n & 1;
       const float* st = stats + s * 256;
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, n & 1, wd, ERR_BWD_S_FULL) &&
@@ -695,7 +753,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                          const CUtensorMap& mdo, const BwdParams& p, cudaStream_t stream,
                          cudaEvent_t ev_begin, cudaEvent_t ev_end) {
@@ -706,7 +764,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: pre kernel launch\n");
     return e;
   }
-  auto kern = bwd_main_kernel<D, CAUSAL>;
+  auto kern = bwd_main_kernel<D, CAUSAL, SPARSE>;
   const int smem = BwdLayout<D>::ALLOC;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) {
@@ -727,14 +785,24 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   return cudaGetLastError();
 }
 
+template <bool SPARSE>
+inline cudaError_t launch_bwd_s(const CUtensorMap& mq, const CUtensorMap& mk,
+                                const CUtensorMap& mv, const CUtensorMap& mdo,
+                                const BwdParams& p, int d, bool causal, cudaStream_t stream,
+                                cudaEvent_t ev_begin, cudaEvent_t ev_end) {
+  if (d == 64)
+    return causal ? launch_bwd_t<64, true, SPARSE>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
+                  : launch_bwd_t<64, false, SPARSE>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
+  return causal ? launch_bwd_t<128, true, SPARSE>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
+                : launch_bwd_t<128, false, SPARSE>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
+}
+
 inline cudaError_t launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                               const CUtensorMap& mdo, const BwdParams& p, int d, bool causal,
                               cudaStream_t stream, cudaEvent_t ev_begin, cudaEvent_t ev_end) {
-  if (d == 64)
-    return causal ? launch_bwd_t<64, true>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
-                  : launch_bwd_t<64, false>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
-  return causal ? launch_bwd_t<128, true>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end)
-                : launch_bwd_t<128, false>(mq, mk, mv, mdo, p, stream, ev_begin, ev_end);
+  return p.bmask != nullptr
+             ? launch_bwd_s<true>(mq, mk, mv, mdo, p, d, causal, stream, ev_begin, ev_end)
+             : launch_bwd_s<false>(mq, mk, mv, mdo, p, d, causal, stream, ev_begin, ev_end);
 }
 
 // One warp waits on an mbarrier that nothing arrives on; the bounded wait

@@ -45,7 +45,16 @@ struct FwdParams {
   int num_qblocks;         // ceil(N / 256)
   float scale_log2;        // scale * log2(e)
   unsigned long long wait_limit_ns;
+  // block-sparse mode only: tile (qt, kt) of sequence b and kv head hk is
+  // allowed iff bmask[b * bm_sb + hk * bm_sh + qt * bm_nt + kt] != 0
+  const uint8_t* bmask;
+  long bm_sb, bm_sh;
+  int bm_nt;
 };
+
+// Largest N of the block-sparse kernels: the per-CTA tile lists live in
+// shared memory.
+constexpr int FA_SPARSE_MAX_TILES = 512;
 
 // Device error word of the library (first error wins; 0 = none).  All
 // kernels live in one translation unit, so one definition serves them all.

@@ -56,7 +56,13 @@ struct FwdLayout {
   // q_full[2] kv_full[NS] kv_empty[NS] s_full[2] s_free[2] p_full[2] p_free[2] drain[1]
   static constexpr int NBAR = 2 + 2 * NS + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int BYTES = OFF_MISC + 16;
+  // block-sparse mode: the CTA's K/V tile list (uint16 [FA_SPARSE_MAX_TILES]),
+  // which Q tile owns each K/V tile (uint32 bits [2][FA_SPARSE_MAX_TILES/32])
+  // and the list's length
+  static constexpr int OFF_LIST = OFF_MISC + 16;
+  static constexpr int OFF_OWN = OFF_LIST + 2 * FA_SPARSE_MAX_TILES;
+  static constexpr int OFF_NLIST = OFF_OWN + 2 * (FA_SPARSE_MAX_TILES / 32) * 4;
+  static constexpr int BYTES = OFF_NLIST + 16;
   static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
 };
 
@@ -79,7 +85,7 @@ constexpr float RESCALE_LOG2 = 8.0f;
 // for the whole pass.)
 constexpr int EXP2_POLY_PAIRS_OF_8 = 0;
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -105,13 +111,44 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   if (q0 >= len) return;
   const int hk = h / p.group;
   const int nkv_all = (len + 127) / 128;
-  int n_t[2];
+  uint16_t* s_list = reinterpret_cast<uint16_t*>(smem + L::OFF_LIST);
+  uint32_t* s_own = reinterpret_cast<uint32_t*>(smem + L::OFF_OWN);
+  int* s_nlist = reinterpret_cast<int*>(smem + L::OFF_NLIST);
+  if (SPARSE && warp == 10) {
+    // Block-sparse: the K/V tiles this CTA streams are those allowed for
+    // either of its two Q tiles (and on or below the diagonal when causal),
+    // in increasing order; a Q tile masks the ones it does not own.
+    const uint8_t* mrow = p.bmask + (long)b * p.bm_sb + (long)hk * p.bm_sh;
+    int cnt = 0;
+    for (int c0 = 0; c0 < nkv_all; c0 += 32) {
+      const int c = c0 + lane;
+      bool own[2];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int r0 = q0 + 128 * t;
-    n_t[t] = (r0 >= len) ? 0 : (CAUSAL ? min(nkv_all, r0 / 128 + 1) : nkv_all);
+      for (int t = 0; t < 2; ++t) {
+        const int qt = 2 * qb + t;
+        own[t] = c < nkv_all && 128 * qt < len && (!CAUSAL || c <= qt) &&
+                 mrow[(long)qt * p.bm_nt + c] != 0;
+      }
+      const uint32_t b0 = __ballot_sync(0xffffffffu, own[0]);
+      const uint32_t b1 = __ballot_sync(0xffffffffu, own[1]);
+      const uint32_t any = b0 | b1;
+      if (lane == 0) {
+        s_own[c0 >> 5] = b0;
+        s_own[FA_SPARSE_MAX_TILES / 32 + (c0 >> 5)] = b1;
+      }
+      if ((any >> lane) & 1u) s_list[cnt + __popc(any & ((1u << lane) - 1u))] = (uint16_t)c;
+      cnt += __popc(any);
+    }
+    if (lane == 0) *s_nlist = cnt;
   }
-  const int nmax = max(n_t[0], n_t[1]);
+  int n_t[2];
+  if (!SPARSE) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int r0 = q0 + 128 * t;
+      n_t[t] = (r0 >= len) ? 0 : (CAUSAL ? min(nkv_all, r0 / 128 + 1) : nkv_all);
+    }
+  }
 
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* ring = smem + L::OFF_RING;
@@ -158,6 +195,14 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{&g_fa_error, abort_flag, p.wait_limit_ns};
+  if (SPARSE) {
+    // both Q tiles step through the whole list (masking the tiles they do
+    // not own), so the dense issue order of the MMA warp applies unchanged
+    const int nl = *s_nlist;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) n_t[t] = (q0 + 128 * t >= len) ? 0 : nl;
+  }
+  const int nmax = max(n_t[0], n_t[1]);
 
   if (warp >= 8) {
   // ============================================================== warpgroup 2
@@ -183,7 +228,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(ring + stage * L::TILE + c * 16384, map, kv_full + stage, c * 64, hk,
-                      seq_start + 128 * (n >> 1), bcoord);
+                      seq_start + 128 * (SPARSE ? (int)s_list[n >> 1] : (n >> 1)), bcoord);
         issued = n + 1;
       }
       if (*abort_flag) {
@@ -235,7 +280,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                    (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = true;
+      // (nmax = 0 only in block-sparse mode, for a CTA with an empty list:
+      // nothing is loaded and nothing issued)
+      bool ok = nmax > 0;
       for (int t = 0; t < 2 && ok; ++t)
         if (n_t[t] > 0) ok = mbar_wait(q_full + t, 0, wd, ERR_FWD_Q_FULL);
       if (ok) ok = mbar_wait(kv_full + 0, 0, wd, ERR_FWD_KV_FULL);
@@ -320,8 +367,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
       }
       // every MMA issued above completes before TMEM can be released
-      mma_commit(drain);
-      mbar_wait_drain(drain, 0, p.wait_limit_ns);
+      if (nmax > 0) {
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0, p.wait_limit_ns);
+      }
     }
     __syncwarp();
   }
@@ -350,10 +399,22 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       tmem_wait_ld32(s + 32);
       tmem_ld32(tS + 64, s + 64);      // second half loads while the first half is scanned
       tmem_ld32(tS + 96, s + 96);
-      // last tile of this Q tile: sequence end and/or causal diagonal mask
-      const bool masked = (j == n - 1);
-      int lim = len - 128 * j;
-      if (CAUSAL) lim = min(lim, qrow + 1 - 128 * j);
+      // last tile of this Q tile: sequence end and/or causal diagonal mask;
+      // block-sparse: any tile may be cut by them, and a tile this Q tile
+      // does not own is masked whole
+      bool masked = (j == n - 1);
+      int lim;
+      if constexpr (SPARSE) {
+        const int kt = s_list[j];
+        const bool own = (s_own[t * (FA_SPARSE_MAX_TILES / 32) + (kt >> 5)] >> (kt & 31)) & 1u;
+        lim = len - 128 * kt;
+        if (CAUSAL) lim = min(lim, qrow + 1 - 128 * kt);
+        if (!own) lim = 0;
+        masked = lim < 128;
+      } else {
+        lim = len - 128 * j;
+        if (CAUSAL) lim = min(lim, qrow + 1 - 128 * j);
+      }
       if (masked) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -463,7 +524,10 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       if (ok) {
         tc_fence_after();
         const bool row_ok = qrow < len;
-        const float inv_l = 1.f / l;
+        // block-sparse: a row whose allowed tiles hold no key has l = 0 and
+        // an all-zero O accumulator; it gets O = 0 and LSE = -inf
+        const bool no_keys = SPARSE && !(l > 0.f);
+        const float inv_l = no_keys ? 0.f : 1.f / l;
         const long tok = (p.cu_seqlens != nullptr) ? (long)seq_start + qrow
                                                     : (long)b * p.N + qrow;
         __nv_bfloat16* orow = p.o + (tok * p.Hq + h) * (long)D;
@@ -485,12 +549,19 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           }
         }
         if (row_ok) {
-          const float lse = (m + log2f(l)) * 0.69314718055994530942f;
+          const float lse = no_keys ? -INFINITY : (m + log2f(l)) * 0.69314718055994530942f;
           const long li = (p.cu_seqlens != nullptr) ? (long)h * p.total + seq_start + qrow
                                                     : ((long)b * p.Hq + h) * p.N + qrow;
           p.lse[li] = lse;
         }
       }
+    } else if (SPARSE && n == 0 && qrow < len) {
+      // no tile allowed for either Q tile of this CTA: nothing was computed
+      const long tok = (long)b * p.N + qrow;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (tok * p.Hq + h) * (long)D);
+#pragma unroll 1
+      for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+      p.lse[((long)b * p.Hq + h) * p.N + qrow] = -INFINITY;
     }
   }
 

@@ -24,7 +24,8 @@ STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
 EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
             "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events",
-            "fa_bwd_noalloc", "fa_std_softmax", "fa_decode", "fa_decode_workspace_size"]
+            "fa_bwd_noalloc", "fa_std_softmax", "fa_decode", "fa_decode_workspace_size",
+            "fa_fwd_blockmask", "fa_bwd_blockmask"]
 
 # capacity of the fixed scratch behind fa_bwd_noalloc (include/fa.h)
 FA_BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -65,6 +66,12 @@ def load(build_if_missing=True):
     lib.fa_bwd.restype = c_int
     lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd_noalloc.restype = c_int
+    cl = ctypes.c_long
+    lib.fa_fwd_blockmask.argtypes = [vp] * 5 + [c_int] * 5 + [c_float, c_int, vp, cl, cl, vp]
+    lib.fa_fwd_blockmask.restype = c_int
+    lib.fa_bwd_blockmask.argtypes = [vp] * 10 + [ctypes.c_size_t] + [c_int] * 5 + \
+        [c_float, c_int, vp, cl, cl, vp]
+    lib.fa_bwd_blockmask.restype = c_int
     lib.fa_decode.argtypes = [vp] * 6 + [c_int] * 5 + [c_float, vp, ctypes.c_size_t, vp]
     lib.fa_decode.restype = c_int
     lib.fa_decode_workspace_size.argtypes = [c_int] * 4
@@ -112,6 +119,19 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, cau
     the library or by this binding); see include/fa.h for its limits."""
     return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
                                  int(causal), cu_seqlens, total_tokens, stream)
+
+
+def fa_fwd_blockmask(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, block_mask, mask_bs,
+                     mask_hs, stream):
+    return load().fa_fwd_blockmask(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, int(causal),
+                                   block_mask, mask_bs, mask_hs, stream)
+
+
+def fa_bwd_blockmask(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N,
+                     d, scale, causal, block_mask, mask_bs, mask_hs, stream):
+    return load().fa_bwd_blockmask(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B,
+                                   Hq, Hkv, N, d, scale, int(causal), block_mask, mask_bs,
+                                   mask_hs, stream)
 
 
 def fa_decode(q, k_cache, v_cache, o, lse, cache_seqlens, B, Hq, Hkv, Lmax, d, scale, workspace,
@@ -269,6 +289,62 @@ class Attention(torch.autograd.Function):
 def attention(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None):
     return Attention.apply(q, k, v, scale if scale is not None else q.shape[-1] ** -0.5,
                            causal, cu_seqlens, max_seqlen)
+
+
+# ------------------------------------------------------------ block-sparse
+
+def _mask_strides(block_mask, B, Hkv, N):
+    _check(block_mask, "block_mask", torch.uint8)
+    nt = (N + 127) // 128
+    if block_mask.dim() != 4 or block_mask.shape[2:] != (nt, nt) or \
+            block_mask.shape[0] not in (1, B) or block_mask.shape[1] not in (1, Hkv):
+        raise ValueError("block_mask must be [1 or B, 1 or Hkv, %d, %d] uint8" % (nt, nt))
+    sb = 0 if block_mask.shape[0] == 1 else block_mask.shape[1] * nt * nt
+    sh = 0 if block_mask.shape[1] == 1 else nt * nt
+    return sb, sh
+
+
+def attention_fwd_blockmask(q, k, v, block_mask, scale=None, causal=False, out=None, lse=None):
+    """O, LSE of block-sparse attention (fa_fwd_blockmask): dense [B, N, H, d]
+    inputs; block_mask [1 or B, 1 or Hkv, nt, nt] uint8 on the device,
+    nt = ceil(N / 128), nonzero = the 128 x 128 tile is computed."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, nm)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    sb, sh = _mask_strides(block_mask, B, Hkv, N)
+    if scale is None:
+        scale = d ** -0.5
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    st = fa_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                          float(scale), causal, _ptr(block_mask), sb, sh, _stream())
+    if st != FA_OK:
+        raise FAError("fa_fwd_blockmask", st)
+    return out, lse
+
+
+def attention_bwd_blockmask(q, k, v, out, lse, dout, block_mask, scale=None, causal=False,
+                            workspace=None):
+    """dQ, dK, dV of block-sparse attention (fa_bwd_blockmask)."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, nm)
+    _check(lse, "lse", torch.float32)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    sb, sh = _mask_strides(block_mask, B, Hkv, N)
+    if scale is None:
+        scale = d ** -0.5
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, Hq, N, d, B * N), dtype=torch.uint8,
+                                device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = fa_bwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                          _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, N,
+                          d, float(scale), causal, _ptr(block_mask), sb, sh, _stream())
+    if st != FA_OK:
+        raise FAError("fa_bwd_blockmask", st)
+    return dq, dk, dv
 
 
 # ------------------------------------------------------------ decode

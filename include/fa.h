@@ -104,6 +104,37 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
 /*
+ * Block-sparse attention: the same forward and backward with every (query,
+ * key) pair removed whose 128 x 128 tile the block mask does not allow -- a
+ * generalisation of causal tile skipping ("FlashAttention优化" 7.2; the
+ * paper review's block-sparse variant); exact on the allowed entries, and
+ * disallowed tiles are never computed.
+ *   block_mask        : device bytes [*][*][nt][nt], nt = ceil(N / 128);
+ *                       tile (qt, kt) of sequence b and key/value head hk is
+ *                       allowed iff block_mask[b * mask_batch_stride +
+ *                       hk * mask_head_stride + qt * nt + kt] != 0
+ *   mask_*_stride     : in elements; 0 uses one mask for all sequences /
+ *                       all key/value heads.  The query heads of a group
+ *                       share their key/value head's mask.
+ * With causal, tiles above the diagonal stay skipped whatever the mask
+ * says.  A query row with no allowed key gets O = 0, LSE = -inf and dQ = 0.
+ * Dense batches only (no cu_seqlens) and N <= 65536 (FA_ERR_UNSUPPORTED
+ * otherwise); every other argument as for fa_fwd / fa_bwd, including the
+ * workspace size (fa_bwd_workspace_size with total_tokens = B * N).
+ */
+fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                           const unsigned char* block_mask, long mask_batch_stride,
+                           long mask_head_stride, cudaStream_t stream);
+
+fa_status fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                           void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                           int N, int d, float scale, int causal,
+                           const unsigned char* block_mask, long mask_batch_stride,
+                           long mask_head_stride, cudaStream_t stream);
+
+/*
  * Capacity, in bytes, of the fixed scratch array behind fa_bwd_noalloc().
  */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES (64u << 20)

@@ -118,3 +118,19 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(args(ws=ctypes.c_void_p(4096 + 16))) == 3
     assert call(args(q=ctypes.c_void_p(4100))) == 1
     assert call(args(B=0)) == 0
+
+
+def test_blockmask_rejects_bad_arguments(lib):
+    p = ctypes.c_void_p(4096)
+    m = ctypes.c_void_p(8192)
+    f = lambda **kw: ops.fa_fwd_blockmask(*([p] * 5), kw.get("B", 1), 2, 2, kw.get("N", 256),
+                                          kw.get("d", 64), 0.125, 0, kw.get("m", m),
+                                          kw.get("sb", 0), kw.get("sh", 0), None)
+    assert f(m=None) == 1
+    assert f(N=65537) == 2          # more tiles than the per-CTA lists hold
+    assert f(d=96) == 2
+    assert f(sb=-1) == 1
+    assert f(B=0) == 0
+    need = ops.fa_bwd_workspace_size(1, 2, 256, 64, 256)
+    g = ops.fa_bwd_blockmask(*([p] * 9), p, need, 1, 2, 2, 256, 64, 0.125, 1, None, 0, 0, None)
+    assert g == 1
