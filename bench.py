@@ -36,6 +36,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("attention fwd+bwd TFLOP/s (bf16, 1×B200) and % of dense BF16 tensor peak")
 DECODE_METRIC = "decode attention over a KV cache: GB/s of K/V cache read (bf16, 1×B200)"
+SPARSE_METRIC = ("block-sparse attention fwd+bwd TFLOP/s on the allowed (query, key) pairs "
+                 "(bf16, 1×B200) and % of dense BF16 tensor peak")
 L2_FLUSH_BYTES = 256 << 20
 DEFAULT_WORKLOAD = "gqa_causal_b2_hq32_hkv8_n4096_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -398,6 +400,92 @@ def source_sha():
     return h.hexdigest()[:16]
 
 
+# ------------------------------------------------------------------ block-sparse
+def run_blocksparse(args, bw):
+    """fa_fwd_blockmask + fa_bwd_blockmask on one GPU; FLOPs counted on the
+    allowed (query, key) pairs only (what the kernels must compute)."""
+    import torch
+    from exact_io_aware_67_b200 import flops, ops, workloads
+    ws, rank, local = dist_env()
+    if ws > 1 or args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": args.impl, "metric": SPARSE_METRIC,
+                              "unavailable": "block-sparse workloads run on one GPU, b200 arm only"}))
+        return 0
+    torch.cuda.set_device(local)
+    w = bw.base
+    inp = workloads.generate(w)
+    mask = workloads.block_mask(bw)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.dout))
+    bm = torch.from_numpy(mask).cuda()
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    o = torch.empty_like(q)
+    wsb = torch.empty(ops.fa_bwd_workspace_size(w.B, w.Hq, w.N, w.d, w.B * w.N),
+                      dtype=torch.uint8, device="cuda")
+    fwd_f = flops.blocksparse_fwd_flops(bw, mask)
+    bwd_f = 2.5 * fwd_f
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            ops.fa_set_profile_events(evs[0], evs[1])
+        ops.attention_fwd_blockmask(q, k, v, bm, w.scale, w.causal, out=o, lse=lse)
+        if evs:
+            ops.fa_set_profile_events(evs[2], evs[3])
+        ops.attention_bwd_blockmask(q, k, v, o, lse, do, bm, w.scale, w.causal, workspace=wsb)
+        if evs:
+            ops.fa_set_profile_events(None, None)
+
+    ops.fa_clear_device_error()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in ev:   # the library records them later; torch must know they exist
+        for e in row:
+            e.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(ev[s_])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if ops.fa_device_error() != 0:
+        raise RuntimeError("device error word 0x%x" % ops.fa_device_error())
+    ms = t0.elapsed_time(t1)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    fwd_tf = fwd_f / (fwd_ms / 1e3) / 1e12
+    bwd_tf = bwd_f / (bwd_ms / 1e3) / 1e12
+    dom, dom_ms, dom_f = (("bwd_main_kernel", bwd_ms, bwd_f) if bwd_ms >= fwd_ms
+                          else ("fwd_kernel", fwd_ms, fwd_f))
+    value = (fwd_f + bwd_f) * args.steps / (ms / 1e3) / 1e12
+    line = {"metric": SPARSE_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 inputs of the workload's shape)",
+            "config": {"workload": bw.name, **bw.describe(),
+                       "allowed_tile_fraction": float(mask.mean()),
+                       "l2": "inputs larger than L2", "parallelism": "1 GPU"},
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_pct_of_peak": 100 * fwd_tf / peak, "bwd_pct_of_peak": 100 * bwd_tf / peak,
+            "roofline": {"bound": "tensor", "kernel": dom,
+                         "achieved": dom_f / (dom_ms / 1e3) / 1e12, "peak": peak,
+                         "unit": "TFLOP/s", "frac": dom_f / (dom_ms / 1e3) / 1e12 / peak,
+                         "traffic": None, "algorithmic_flops_per_launch": dom_f,
+                         "avg_launch_ms": dom_ms, "peak_source": "%s bf16_tflops (burst)" % src},
+            "gpu_launches": 4 * args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ decode
 def decode_bytes(w, lengths):
     """Algorithmic bytes of one decode step: every valid K and V cache row
@@ -602,6 +690,8 @@ def main():
     from exact_io_aware_67_b200 import workloads
     if args.workload in workloads.DECODE_WORKLOADS:
         return run_decode(args, workloads.DECODE_WORKLOADS[args.workload], args.impl)
+    if args.workload in workloads.BLOCKSPARSE_WORKLOADS:
+        return run_blocksparse(args, workloads.BLOCKSPARSE_WORKLOADS[args.workload])
     w = workloads.WORKLOADS[args.workload]
     if args.warmup < 3 and args.impl == "b200":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

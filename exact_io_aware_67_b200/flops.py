@@ -62,3 +62,37 @@ def bwd_bytes(w, lengths=None):
                   + e * (qh + 2 * kh)          # dq, dk, dv written
                   + 4 * w.Hq * 2               # lse read, D written
                   + 4 * qh * 3)                # dq_acc zero, reduce, read
+
+
+def blocksparse_pairs(N, causal, mask_row):
+    """(query, key) pairs a block mask allows in one head: the sum over the
+    allowed 128 x 128 tiles of their element count, cut at N, and with only
+    j <= i kept on diagonal tiles when causal (off-diagonal allowed tiles
+    below it count whole; tiles above it are never allowed)."""
+    import numpy as np
+    m = np.asarray(mask_row, dtype=bool)
+    nt = m.shape[0]
+    sizes = np.minimum(128, N - 128 * np.arange(nt))
+    total = 0
+    for qt in range(nt):
+        for kt in range(nt):
+            if not m[qt, kt] or (causal and kt > qt):
+                continue
+            if causal and kt == qt:
+                r = int(sizes[qt])
+                total += r * (r + 1) // 2
+            else:
+                total += int(sizes[qt]) * int(sizes[kt])
+    return total
+
+
+def blocksparse_fwd_flops(bw, mask):
+    """4 d per allowed (query, key) pair, summed over query heads (each uses
+    its key/value head's mask row)."""
+    w = bw.base
+    g = w.Hq // w.Hkv
+    tot = 0
+    for hk in range(w.Hkv):
+        row = mask[0, hk if mask.shape[1] > 1 else 0]
+        tot += g * blocksparse_pairs(w.N, w.causal, row)
+    return 4.0 * w.d * tot * w.B

@@ -224,3 +224,54 @@ def generate_decode(w: DecodeWorkload) -> DecodeInputs:
     v = torch.randn((w.B, w.Lmax, w.Hkv, w.d), generator=g, dtype=torch.float32)
     bf = torch.bfloat16
     return DecodeInputs(q=q.to(bf), k=k.to(bf), v=v.to(bf), seqlens=seqlens, workload=w)
+
+
+# ------------------------------------------------------------ block-sparse masks
+
+@dataclass
+class BlockSparseWorkload:
+    """A dense workload plus a block mask of 128 x 128 tiles: ``band`` = w
+    keeps the w tiles on and left of the diagonal (a sliding window of 128 w
+    keys), ``density`` = r keeps each tile with probability r (per kv head,
+    drawn from the workload's seed after its inputs), the diagonal always."""
+    name: str
+    base: Workload
+    band: Optional[int] = None
+    density: Optional[float] = None
+
+    def describe(self):
+        out = dict(self.base.describe())
+        if self.band is not None:
+            out["block_mask"] = "band of %d tiles (%d keys)" % (self.band, 128 * self.band)
+        else:
+            out["block_mask"] = "random tiles, density %.2f per kv head, diagonal kept" % self.density
+        return out
+
+
+def block_mask(bw: BlockSparseWorkload):
+    """uint8 [1, 1 or Hkv, nt, nt] mask of the workload."""
+    import numpy as np
+    w = bw.base
+    nt = (w.N + 127) // 128
+    i = np.arange(nt)
+    if bw.band is not None:
+        m = ((i[:, None] - i[None, :] >= 0) & (i[:, None] - i[None, :] < bw.band))
+        return m.astype(np.uint8)[None, None]
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 1000003)
+    m = (torch.rand((1, w.Hkv, nt, nt), generator=g) < bw.density).numpy()
+    m[:, :, i, i] = True
+    return m.astype(np.uint8)
+
+
+BLOCKSPARSE_WORKLOADS = {
+    # a causal sliding window of 1024 keys over a 16384-token sequence
+    "blocksparse_band8_causal_b1_h16_n16384_d128": BlockSparseWorkload(
+        "blocksparse_band8_causal_b1_h16_n16384_d128",
+        _w("blocksparse_band8_causal_b1_h16_n16384_d128", 1, 16, 16384, 128, True), band=8),
+    # random half of the tiles of a non-causal 8192-token problem, GQA 4
+    "blocksparse_random50_b1_hq16_hkv4_n8192_d64": BlockSparseWorkload(
+        "blocksparse_random50_b1_hq16_hkv4_n8192_d64",
+        _w("blocksparse_random50_b1_hq16_hkv4_n8192_d64", 1, 16, 8192, 64, False, Hkv=4),
+        density=0.5),
+}

@@ -108,3 +108,25 @@ def test_blockmask_band_long_sequence():
     bm = ((i[:, None] - i[None, :] >= 0) & (i[:, None] - i[None, :] < 4)).astype(np.uint8)
     bm = bm[None, None]
     _check(inp, bm, True, _run(inp, bm, True))
+
+
+@pytest.mark.parametrize("name", sorted(workloads.BLOCKSPARSE_WORKLOADS))
+def test_blocksparse_workloads_first_group(name):
+    # the benchmark's block-sparse workloads at full size; the oracle checks
+    # every output of kv head 0's query heads (and kv head 0's dK, dV)
+    bw = workloads.BLOCKSPARSE_WORKLOADS[name]
+    w = bw.base
+    inp = workloads.generate(w)
+    bm = workloads.block_mask(bw)
+    o, lse, dq, dk, dv = _run(inp, bm, w.causal)
+    g = w.Hq // w.Hkv
+    f = lambda t: t.double().numpy()
+    sub = lambda t, n: np.ascontiguousarray(f(t)[:, :, :n])
+    ref = oracle.attention_bwd_blockmask(sub(inp.q, g), sub(inp.k, 1), sub(inp.v, 1),
+                                         sub(inp.dout, g), w.scale, w.causal, bm[:, :1])
+    parity.assert_close("O", parity.f64(o[:, :, :g]), ref["o"])
+    parity.assert_close("LSE", parity.f64(lse[:, :g]), ref["lse"], tol_max=parity.TOL_LSE,
+                        tol_mean=None, bf16_out=False)
+    parity.assert_close("dQ", parity.f64(dq[:, :, :g]), ref["dq"])
+    parity.assert_close("dK", parity.f64(dk[:, :, :1]), ref["dk"])
+    parity.assert_close("dV", parity.f64(dv[:, :, :1]), ref["dv"])
