@@ -419,13 +419,17 @@ fa_status fa_decode(const void* q, const void* k_cache, const void* v_cache, voi
   p.Hkv = Hkv;
   p.Lmax = Lmax;
   p.group = Hq / Hkv;
-  fa::decode_plan(B, Hkv, Lmax, sms, &p.chunk, &p.splits);
-  if ((long long)B * Hkv * p.splits > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  p.items = B * Hkv * p.splits;
-  const size_t o_bytes = (size_t)p.splits * B * Hq * d * 4;
-  p.o_part = static_cast<float*>(workspace);
-  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                        ((o_bytes + 255) & ~(size_t)255));
+  // one CTA per SM (at most the number of tiles when every cache is full;
+  // with device-side lengths some CTAs may get empty ranges)
+  const long long tiles_full = (long long)B * Hkv * ((Lmax + 127) / 128);
+  p.grid = (int)std::min<long long>(std::min(sms, fa::DEC_MAX_GRID), tiles_full);
+  char* wsp = static_cast<char*>(workspace);
+  p.boff = reinterpret_cast<long long*>(wsp);
+  wsp += ((size_t)(B + 1) * 8 + 255) & ~(size_t)255;
+  const size_t rows = (size_t)B * Hq + (size_t)fa::DEC_MAX_GRID * fa::DEC_GMAX;
+  p.o_part = reinterpret_cast<float*>(wsp);
+  wsp += (rows * d * 4 + 255) & ~(size_t)255;
+  p.lse_part = reinterpret_cast<float*>(wsp);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit_ns = g_wait_limit_ns.load();
   e = fa::launch_decode(mk, mv, p, d, stream);

@@ -10,14 +10,16 @@
 // not by arithmetic -- about 2 FLOP per byte of K and V at Hq/Hkv = 1.
 //
 // B200 design:
-//  * Split-KV.  The cache of each (sequence, kv head) is cut into chunks of
-//    `chunk` keys and every chunk is its own CTA, so that a few sequences
-//    still fill 148 SMs.  A CTA serves all g = Hq/Hkv query heads of its kv
-//    head, so each K and V element leaves HBM once.  It writes a partial
-//    (o_s normalised by its own sum, lse_s) to the workspace; the merge
-//    kernel combines the chunks exactly: lse = ln sum_s e^(lse_s) and
-//    o = sum_s e^(lse_s - lse) o_s (the online-softmax merge rule of the
-//    blog post's 3.2.1, applied to chunk results).
+//  * Split-KV, balanced.  The 128-key tiles of every (sequence, kv head)
+//    pair, laid end to end, are cut into one contiguous range per CTA of
+//    equal length (to one tile), so that a few long caches or many short
+//    ones fill the 148 SMs alike.  A CTA serves all g = Hq/Hkv query heads
+//    of a kv head, so each K and V element leaves HBM once.  For every pair
+//    its range touches it writes a partial (o_s normalised by its own sum,
+//    lse_s); the merge kernel combines each pair's partials exactly:
+//    lse = ln sum_s e^(lse_s) and o = sum_s e^(lse_s - lse) o_s (the
+//    online-softmax merge rule of the blog post's 3.2.1, applied to chunk
+//    results).
 //  * K and V tiles of 128 keys move by TMA (the same token-major tensor maps
 //    as the training kernels) into a two-stage shared-memory ring; thread 0
 //    refills a stage once every thread has passed the tile's last barrier.
@@ -46,13 +48,16 @@ struct DecodeParams {
   __nv_bfloat16* o;         // [B][Hq][D]
   float* lse;               // [B][Hq]
   const int* seqlens;       // [B] cached keys per sequence, or null (all Lmax)
-  float* o_part;            // [splits][B][Hq][D]  chunk outputs, normalised
-  float* lse_part;          // [splits][B][Hq]     chunk LSE (natural log)
-  int B, Hq, Hkv, Lmax, group, chunk, splits;
-  int items;                // B * Hkv * splits work items (sequence, kv head, chunk)
+  long long* boff;          // [B + 1] tiles of the sequences before b (with seqlens)
+  float* o_part;            // [B * Hkv + grid][g][D] range partials, normalised
+  float* lse_part;          // [B * Hkv + grid][g]    their LSE (natural log)
+  int B, Hq, Hkv, Lmax, group;
+  int grid;                 // CTAs of the split kernel
   float scale_log2;
   unsigned long long wait_limit_ns;
 };
+
+constexpr int DEC_MAX_GRID = 1024;   // bound used by the workspace size
 
 constexpr int DEC_CONSUMERS = 8;                     // warps that compute
 constexpr int DEC_THREADS = 32 * (DEC_CONSUMERS + 1);  // + one TMA producer warp
@@ -74,25 +79,79 @@ struct DecodeLayout {
   static_assert(ALLOC <= 227 * 1024, "shared memory per block");
 };
 
-// Work item i: chunk (i mod splits) of kv head hk of sequence b, with
-// i / splits = b * Hkv + hk.  Its keys are [k0, k1).
-struct DecodeItem {
-  int b, hk, split, k0, k1, ntiles;
+// Tiles of sequence b, and the tiles of the sequences before it (per kv
+// head): the flattened tile space is pair-major, pair = b * Hkv + hk.
+__device__ __forceinline__ int dec_len(const DecodeParams& p, int b) {
+  return p.seqlens != nullptr ? min(max(p.seqlens[b], 0), p.Lmax) : p.Lmax;
+}
+__device__ __forceinline__ int dec_ntiles(const DecodeParams& p, int b) {
+  return (dec_len(p, b) + DEC_TILE - 1) / DEC_TILE;
+}
+__device__ __forceinline__ long long dec_boff(const DecodeParams& p, int b) {
+  return p.seqlens != nullptr ? p.boff[b]
+                              : (long long)b * ((p.Lmax + DEC_TILE - 1) / DEC_TILE);
+}
+__device__ __forceinline__ long long dec_total(const DecodeParams& p) {
+  return (long long)p.Hkv * dec_boff(p, p.B);
+}
+// first flattened tile of CTA c's range: floor(c T / grid)
+__device__ __forceinline__ long long dec_range_start(long long c, long long T, int grid) {
+  return c * T / grid;
+}
+// the CTA whose range holds flattened tile x
+__device__ __forceinline__ int dec_cta_of(long long x, long long T, int grid) {
+  return (int)(((x + 1) * grid - 1) / T);
+}
+
+// One contiguous piece of a CTA's range inside one (sequence, kv head) pair.
+struct DecodeSeg {
+  int b, hk, k0, k1, ntiles;
+  long long slot;   // partial slot: pair + CTA (unique, increasing along the ranges)
 };
 
-__device__ __forceinline__ DecodeItem decode_item(const DecodeParams& p, int i) {
-  DecodeItem it;
-  it.split = i % p.splits;
-  const int pair = i / p.splits;
-  it.hk = pair % p.Hkv;
-  it.b = pair / p.Hkv;
-  int len = p.Lmax;
-  if (p.seqlens != nullptr) len = min(max(p.seqlens[it.b], 0), p.Lmax);
-  it.k0 = it.split * p.chunk;
-  it.k1 = min(it.k0 + p.chunk, len);
-  it.ntiles = (it.k1 > it.k0) ? (it.k1 - it.k0 + DEC_TILE - 1) / DEC_TILE : 0;
-  return it;
-}
+// Walks a CTA's range [pos, end) pair by pair.
+struct DecodeWalker {
+  int b, hk, tile;
+  long long pos, end;
+
+  __device__ void init(const DecodeParams& p, long long t0, long long t1) {
+    pos = t0;
+    end = t1;
+    if (pos >= end) return;
+    // the sequence whose tiles hold t0: largest b with Hkv * boff(b) <= t0
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((long long)p.Hkv * dec_boff(p, mid) <= t0) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    const int nt = dec_ntiles(p, b);
+    const long long r = t0 - (long long)p.Hkv * dec_boff(p, b);
+    hk = (int)(r / nt);
+    tile = (int)(r % nt);
+  }
+  __device__ bool next(const DecodeParams& p, DecodeSeg& sg) {
+    if (pos >= end) return false;
+    const int nt = dec_ntiles(p, b);
+    const int n = (int)min((long long)(nt - tile), end - pos);
+    sg.b = b;
+    sg.hk = hk;
+    sg.k0 = tile * DEC_TILE;
+    sg.k1 = min((tile + n) * DEC_TILE, dec_len(p, b));
+    sg.ntiles = n;
+    sg.slot = (long long)b * p.Hkv + hk + blockIdx.x;
+    pos += n;
+    tile = 0;
+    if (++hk == p.Hkv) {
+      hk = 0;
+      do {
+        ++b;
+      } while (b < p.B && dec_ntiles(p, b) == 0);
+    }
+    return true;
+  }
+};
 
 // 16 x 8 x 16 bf16 MMA with fp32 accumulation (sm_80+ warp-level form; the
 // query heads of one kv head are at most 16 rows, the M of this shape).
@@ -120,12 +179,12 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int r, int c) {
                            ((((c & 63) >> 3) ^ (r & 7)) << 4));
 }
 
-// Persistent: gridDim.x CTAs (at most one per SM) take the items
-// blockIdx.x, blockIdx.x + gridDim.x, ...  Warp 8 streams their K and V
-// tiles through the TMA ring, across item boundaries; warps 0-7 each take
-// 16 keys of every tile with their own online-softmax state (running max
-// and sum per query head, and a 16 x D output fragment), and merge the
-// eight states when an item ends.
+// Persistent: gridDim.x CTAs (at most one per SM), each with one contiguous
+// range of the flattened tiles.  Warp 8 streams the range's K and V tiles
+// through the TMA ring, across pair boundaries; warps 0-7 each take 16 keys
+// of every tile with their own online-softmax state (running max and sum
+// per query head, and a 16 x D output fragment), and merge the eight states
+// at the end of each pair's piece.
 //
 // Per warp and tile: S^T = Q K^T as (heads x 16 keys), Q held in registers
 // as MMA A-fragments for the whole item and K^T fragments read with
@@ -144,6 +203,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   uint8_t* smem = align_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = p.group;
+  const long long T = dec_total(p);   // tiles of the whole batch, per kv head summed
 
   uint8_t* ring = smem + L::OFF_KV;
   float* sr = reinterpret_cast<float*>(smem + L::OFF_R);
@@ -173,8 +233,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       tma_prefetch_desc(&tmV);
       long c = 0;   // stream position
       bool pok = true;
-      for (int item = blockIdx.x; pok && item < p.items; item += gridDim.x) {
-        const DecodeItem it = decode_item(p, item);
+      DecodeWalker wk;
+      DecodeSeg it;
+      wk.init(p, dec_range_start(blockIdx.x, T, gridDim.x),
+              dec_range_start(blockIdx.x + 1, T, gridDim.x));
+      while (pok && wk.next(p, it)) {
         for (int t = 0; pok && t < it.ntiles; ++t, ++c) {
           const int st = (int)(c % ST);
           if (c >= ST && !(pok = mbar_wait(empty + st, (uint32_t)((c / ST - 1) & 1), wd,
@@ -208,17 +271,14 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   long c = 0;                        // stream position
   bool ok = true;
 
-  for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
-    const DecodeItem it = decode_item(p, item);
+  DecodeWalker wk;
+  DecodeSeg it;
+  wk.init(p, dec_range_start(blockIdx.x, T, gridDim.x),
+          dec_range_start(blockIdx.x + 1, T, gridDim.x));
+  while (wk.next(p, it)) {
     const int h0 = it.hk * g;
-    float* opart = p.o_part + (((long)it.split * p.B + it.b) * p.Hq + h0) * D;
-    float* lpart = p.lse_part + ((long)it.split * p.B + it.b) * p.Hq + h0;
-    if (it.ntiles == 0) {
-      // nothing cached in this chunk: the merge's neutral element
-      for (int i = tid; i < g * D; i += 32 * DEC_CONSUMERS) opart[i] = 0.f;
-      for (int i = tid; i < g; i += 32 * DEC_CONSUMERS) lpart[i] = -INFINITY;
-      continue;
-    }
+    float* opart = p.o_part + it.slot * g * D;
+    float* lpart = p.lse_part + it.slot * g;
     // Q of the group as A-fragments (rows = heads, zero past g)
     uint32_t qa[KS][4];
     {
@@ -387,64 +447,96 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   }
 }
 
-// Merge the chunk partials of one (sequence, query head): grid B * Hq, D
-// threads (one output column each).  The chunk weights e^(lse_s - max) go
-// through shared memory D at a time, so that every thread's sum over the
-// chunks is a run of independent loads.
+// Merge the partials of one (sequence, query head): grid B * Hq, D threads
+// (one output column each).  The pair's partials sit in the slots pair + c
+// of the CTAs c whose ranges overlap its tiles.  Their weights e^(lse_s -
+// max) go through shared memory D at a time, so that every thread's sum is
+// a run of independent loads.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
   __shared__ float wsh[D];
   __shared__ float red[D / 32];
-  const long bh = blockIdx.x;   // b * Hq + h
-  const long stride = (long)p.B * p.Hq;
+  const int bh = blockIdx.x;   // b * Hq + h
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int g = p.group, hk = h / g, hg = h - hk * g;
   const int tid = threadIdx.x;
-  float mx = -INFINITY;
-  for (int s = tid; s < p.splits; s += D) mx = fmaxf(mx, p.lse_part[s * stride + bh]);
+  const int nt = dec_ntiles(p, b);
+  float acc = 0.f, wsum = 0.f, M = -INFINITY;
+  if (nt > 0) {
+    const long long T = dec_total(p);
+    const long long off = (long long)p.Hkv * dec_boff(p, b) + (long long)hk * nt;
+    const int c0 = dec_cta_of(off, T, p.grid), c1 = dec_cta_of(off + nt - 1, T, p.grid);
+    const int ns = c1 - c0 + 1;
+    const long long s0 = (long long)b * p.Hkv + hk + c0;   // first slot
+    // a CTA between c0 and c1 with an empty range (more CTAs than tiles)
+    // wrote no partial: it is skipped
+    auto has_range = [&](int c) {
+      return dec_range_start(c, T, p.grid) < dec_range_start(c + 1, T, p.grid);
+    };
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += D)
+      if (has_range(c0 + s)) mx = fmaxf(mx, p.lse_part[(s0 + s) * g + hg]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((tid & 31) == 0) red[tid >> 5] = mx;
-  __syncthreads();
-  float M = -INFINITY;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
-  float acc = 0.f, wsum = 0.f;
-  if (M != -INFINITY) {
-    for (int s0 = 0; s0 < p.splits; s0 += D) {
-      const int n = min(D, p.splits - s0);
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
+    for (int sb = 0; sb < ns; sb += D) {
+      const int n = min(D, ns - sb);
       __syncthreads();
-      if (tid < n) wsh[tid] = expf(p.lse_part[(s0 + tid) * stride + bh] - M);
+      if (tid < n)
+        wsh[tid] = has_range(c0 + sb + tid) ? expf(p.lse_part[(s0 + sb + tid) * g + hg] - M)
+                                            : -1.f;   // no partial
       __syncthreads();
-      const float* op = p.o_part + ((s0 * stride) + bh) * D + tid;
+      const float* op = p.o_part + ((s0 + sb) * g + hg) * D + tid;
 #pragma unroll 8
       for (int k = 0; k < n; ++k) {
         const float w = wsh[k];
-        wsum += w;
-        acc = fmaf(w, op[k * stride * D], acc);
+        if (w >= 0.f) {
+          wsum += w;
+          acc = fmaf(w, op[(long long)k * g * D], acc);
+        }
       }
     }
     acc /= wsum;
   }
-  p.o[bh * D + tid] = __float2bfloat16_rn(acc);
-  if (tid == 0) p.lse[bh] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
+  p.o[(long long)bh * D + tid] = __float2bfloat16_rn(acc);
+  if (tid == 0) p.lse[bh] = (nt == 0) ? -INFINITY : M + logf(wsum);
 }
 
-// Chunking: about four items per SM over the whole batch, each at least
-// one 128-key tile and at most a whole cache, so that the static assignment
-// of equal items to persistent CTAs balances while the per-item work (q
-// fragments, the merge of the warps' states, the partial's write) and the
-// number of partials stay small.
-inline void decode_plan(int B, int Hkv, int Lmax, int sms, int* chunk, int* splits) {
-  const long tiles = (Lmax + DEC_TILE - 1) / DEC_TILE;
-  const long total = tiles * B * Hkv;
-  const long per_item = std::max(1L, std::min(tiles, (total + 4L * sms - 1) / (4L * sms)));
-  *chunk = (int)(per_item * DEC_TILE);
-  *splits = (Lmax + *chunk - 1) / *chunk;
+// Tiles before each sequence (exclusive prefix sum of ceil(L_b / 128)), one
+// block: needed when the cache lengths live on the device.
+__global__ void __launch_bounds__(1024) decode_prefix_kernel(const DecodeParams p) {
+  __shared__ long long part[1024];
+  const int tid = threadIdx.x;
+  const int per = (p.B + 1023) / 1024;
+  const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+  long long sum = 0;
+  for (int b = b0; b < b1; ++b) sum += dec_ntiles(p, b);
+  part[tid] = sum;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {   // inclusive scan
+    const long long v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  long long run = part[tid] - sum;   // exclusive
+  for (int b = b0; b < b1; ++b) {
+    p.boff[b] = run;
+    run += dec_ntiles(p, b);
+  }
+  if (tid == 1023) p.boff[p.B] = part[1023];
 }
 
 inline size_t decode_workspace_bytes(int B, int Hq, int Lmax, int d) {
-  const size_t splits = (size_t)((Lmax + DEC_TILE - 1) / DEC_TILE);   // upper bound
-  const size_t o = splits * B * Hq * d * 4;
-  return ((o + 255) & ~(size_t)255) + ((splits * B * Hq * 4 + 255) & ~(size_t)255);
+  (void)Lmax;
+  const size_t boff = ((size_t)(B + 1) * 8 + 255) & ~(size_t)255;
+  // slots (B * Hkv + grid) x g heads <= B * Hq + grid * 16
+  const size_t rows = (size_t)B * Hq + (size_t)DEC_MAX_GRID * DEC_GMAX;
+  const size_t o = (rows * d * 4 + 255) & ~(size_t)255;
+  return boff + o + ((rows * 4 + 255) & ~(size_t)255);
 }
 
 template <int D>
@@ -454,14 +546,16 @@ cudaError_t launch_decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
   const int smem = DecodeLayout<D>::ALLOC;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)std::min(p.items, sms);
-  kern<<<grid, DEC_THREADS, smem, stream>>>(mk, mv, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (p.seqlens != nullptr) {
+    decode_prefix_kernel<<<1, 1024, 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.grid > 0) {
+    kern<<<(unsigned)p.grid, DEC_THREADS, smem, stream>>>(mk, mv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   decode_merge_kernel<D><<<(unsigned)(p.B * p.Hq), D, 0, stream>>>(p);
   return cudaGetLastError();
 }

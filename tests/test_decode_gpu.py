@@ -87,6 +87,8 @@ def _custom(B, Hq, Hkv, Lmax, d, lengths=None, seed=0):
     (2, 2, 2, 640, 128, [0, 640]),              # an empty cache
     (40, 8, 8, 200, 64, None),                  # enough CTAs for a single chunk
     (2, 4, 1, 5000, 64, [4999, 3000]),          # one kv head, long ragged caches
+    (2, 4, 1, 1280, 64, [1280, 1]),             # more CTAs than tiles: empty ranges
+    (3, 8, 8, 4096, 128, [0, 3000, 0]),         # empty sequences around a long one
 ])
 def test_decode_matches_oracle(B, Hq, Hkv, Lmax, d, lengths):
     inp = _custom(B, Hq, Hkv, Lmax, d, lengths, seed=Lmax)
