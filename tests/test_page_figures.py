@@ -72,3 +72,29 @@ def test_generator_is_deterministic_and_ordered():
     iv = workloads.generate(wv)
     assert len(iv.lengths) == 32 and all(128 <= L <= 512 for L in iv.lengths)
     assert int(iv.cu_seqlens[-1]) == sum(iv.lengths) == iv.q.shape[0]
+
+
+# ------------------------------------------------- block-sparse accounting
+
+@pytest.mark.parametrize("N,causal,seed", [(300, False, 1), (300, True, 2), (1024, True, 3),
+                                           (1000, False, 4)])
+def test_blocksparse_pairs_match_brute_force(N, causal, seed):
+    # allowed (query, key) pairs of a block mask, counted element by element
+    import numpy as np
+    nt = (N + 127) // 128
+    rng = np.random.default_rng(seed)
+    m = rng.random((nt, nt)) < 0.5
+    el = np.repeat(np.repeat(m, 128, axis=0), 128, axis=1)[:N, :N]
+    if causal:
+        el &= np.tril(np.ones((N, N), dtype=bool))
+    assert flops.blocksparse_pairs(N, causal, m) == int(el.sum())
+
+
+def test_blocksparse_flops_all_allowed_equals_dense_count():
+    # with every tile allowed and no mask, 4 d per pair over all N^2 pairs is
+    # the dense forward count
+    import numpy as np
+    bw = workloads.BlockSparseWorkload(
+        "t", workloads.custom("t", 2, 4, 2, 512, 64, False), density=1.0)
+    mask = np.ones((1, 2, 4, 4), dtype=np.uint8)
+    assert flops.blocksparse_fwd_flops(bw, mask) == flops.fwd_flops(bw.base)
