@@ -7,7 +7,7 @@
 // over keys 0..L_b-1, and lse = ln sum_j exp(scale q.k_j).  The tutorial's
 // 2.3.1 and the blog post's 4.2 describe this decode step: every generated
 // token re-reads the whole cache, so the step is bound by HBM bandwidth,
-// not by arithmetic -- about 2 FLOP per byte of K and V at Hq/Hkv = 1.
+// not by arithmetic -- about 2 FLOP per byte of K and V per query head.
 //
 // B200 design:
 //  * Split-KV, balanced.  The 128-key tiles of every (sequence, kv head)
@@ -20,23 +20,17 @@
 //    lse = ln sum_s e^(lse_s) and o = sum_s e^(lse_s - lse) o_s (the
 //    online-softmax merge rule of the blog post's 3.2.1, applied to chunk
 //    results).
-//  * K and V tiles of 128 keys move by TMA (the same token-major tensor maps
-//    as the training kernels) into a two-stage shared-memory ring; thread 0
-//    refills a stage once every thread has passed the tile's last barrier.
-//  * S: a thread owns one key and half of the query heads; its K row is read
-//    from the 128-byte-swizzled tile (conflict-free) and dotted with q, held
-//    in shared memory in fp32 and pre-scaled by scale * log2(e).
-//  * Online softmax per tile in exp2: tile max per head (one warp per head),
-//    running max m and the rescale factor in shared memory, p written back
-//    over s.
-//  * PV: a warp owns 16 keys of the tile and a lane owns D/32 output columns
-//    for every head, so each V element is converted once per CTA and the
-//    probabilities are shared-memory broadcasts.  The eight warps' partial
-//    outputs are summed once per chunk.
-//  * Arithmetic on CUDA cores: at g <= 8 the FMA work stays under the time
-//    the K/V bytes take to arrive, so the tensor cores buy nothing here.
-//  * Keys at or past L_b are masked (their cache rows may hold anything);
-//    chunks that start past L_b write the merge's neutral element.
+//  * One TMA producer warp streams the range's K and V tiles through a
+//    shared-memory ring, across pair boundaries; eight consumer warps take
+//    16 keys of every tile each, with S = Q K^T and O += P V as m16n8k16
+//    bf16 tensor-core products (the g query heads are the 16 MMA rows, q
+//    stays in registers, and the fp32 S fragment is P's A fragment).
+//  * Keys at or past L_b are masked (their cache rows may hold anything).
+//  * Launches: [prefix kernel, when the lengths live on the device,] split
+//    kernel, merge kernel.  The split and merge kernels are programmatic
+//    dependent launches: their CTAs become resident and run their set-up
+//    while the previous kernel finishes, then wait for it (griddep_wait)
+//    before their first read or write of global memory.
 #pragma once
 #include "fa_common.cuh"
 #include "sm100.cuh"
@@ -127,6 +121,10 @@ struct DecodeWalker {
     }
     b = lo;
     const int nt = dec_ntiles(p, b);
+    if (nt == 0) {   // only if the offsets disagreed with the lengths
+      pos = end;
+      return;
+    }
     const long long r = t0 - (long long)p.Hkv * dec_boff(p, b);
     hk = (int)(r / nt);
     tile = (int)(r % nt);
@@ -152,6 +150,18 @@ struct DecodeWalker {
     return true;
   }
 };
+
+// Programmatic dependent launch.  griddep_wait blocks until the grids this
+// one depends on have completed and their writes are visible; launched
+// without the attribute, stream order has already done that and it returns
+// at once.  griddep_launch_dependents lets the next kernel's CTAs start
+// their own set-up (they wait in the same way before touching memory).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // 16 x 8 x 16 bf16 MMA with fp32 accumulation (sm_80+ warp-level form; the
 // query heads of one kv head are at most 16 rows, the M of this shape).
@@ -203,7 +213,6 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   uint8_t* smem = align_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = p.group;
-  const long long T = dec_total(p);   // tiles of the whole batch, per kv head summed
 
   uint8_t* ring = smem + L::OFF_KV;
   float* sr = reinterpret_cast<float*>(smem + L::OFF_R);
@@ -224,13 +233,21 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   }
   for (int i = tid; i < DEC_GMAX * D; i += DEC_THREADS) sr[i] = 0.f;
   for (int i = tid; i < DEC_GMAX; i += DEC_THREADS) sl[i] = 0.f;
+  if (warp == DEC_CONSUMERS && lane == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
   __syncthreads();
+  if (tid == 0) griddep_launch_dependents();
+  // Nothing above touched global memory.  From here on the kernel reads
+  // the lengths, the tile offsets, q and the caches, and writes the
+  // partials that the previous call's merge kernel may still be reading.
+  griddep_wait();
+  const long long T = dec_total(p);   // tiles of the whole batch, per kv head summed
 
   if (warp == DEC_CONSUMERS) {
     // ============================================================ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
       long c = 0;   // stream position
       bool pok = true;
       DecodeWalker wk;
@@ -460,6 +477,7 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int g = p.group, hk = h / g, hg = h - hk * g;
   const int tid = threadIdx.x;
+  griddep_wait();   // the split kernel's partials (and, before it, the offsets)
   const int nt = dec_ntiles(p, b);
   float acc = 0.f, wsum = 0.f, M = -INFINITY;
   if (nt > 0) {
@@ -510,6 +528,7 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
 __global__ void __launch_bounds__(1024) decode_prefix_kernel(const DecodeParams p) {
   __shared__ long long part[1024];
   const int tid = threadIdx.x;
+  if (tid == 0) griddep_launch_dependents();   // the split kernel waits for our writes
   const int per = (p.B + 1023) / 1024;
   const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
   long long sum = 0;
@@ -551,13 +570,24 @@ cudaError_t launch_decode_d(const CUtensorMap& mk, const CUtensorMap& mv, const 
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
   if (p.grid > 0) {
-    kern<<<(unsigned)p.grid, DEC_THREADS, smem, stream>>>(mk, mv, p);
-    e = cudaGetLastError();
+    cfg.gridDim = dim3((unsigned)p.grid);
+    cfg.blockDim = dim3(DEC_THREADS);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    e = cudaLaunchKernelEx(&cfg, kern, mk, mv, p);
     if (e != cudaSuccess) return e;
   }
-  decode_merge_kernel<D><<<(unsigned)(p.B * p.Hq), D, 0, stream>>>(p);
-  return cudaGetLastError();
+  cfg.gridDim = dim3((unsigned)(p.B * p.Hq));
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<D>, p);
 }
 
 inline cudaError_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
