@@ -418,20 +418,27 @@ def load_traffic(kernel, workload):
         ent = d.get(kernel, {}).get(workload)
         if not ent:
             return None
-        if ent.get("source_sha") != source_sha():
+        if kernel not in KERNEL_SOURCES or ent.get("source_sha") != source_sha(kernel):
             return None
         return ent.get("dram_bytes_per_launch")
     except Exception:
         return None
 
 
-def source_sha():
+# the sources a kernel's DRAM traffic depends on: its own header, the shared
+# helpers, and the host file that sets its launch configuration
+KERNEL_SOURCES = {
+    "fwd_kernel": ("fa_fwd.cuh", "fa_common.cuh", "sm100.cuh", "fa_api.cu"),
+    "bwd_main_kernel": ("fa_bwd.cuh", "fa_common.cuh", "sm100.cuh", "fa_api.cu"),
+}
+
+
+def source_sha(kernel):
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_67_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
