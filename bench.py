@@ -696,12 +696,15 @@ def run_decode(args, w, impl):
                    "l2": ("flushed between timed steps (256 MB write)" if flush_l2 else
                           "cache larger than twice the L2 (%.0f MB per step)" % (step_bytes / 1e6)),
                    "parallelism": "independent batches per GPU" if ws > 1 else "1 GPU"},
-        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + decode_merge_kernel",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("decode_split_kernel + decode_merge_kernel" if sl is None else
+                                "decode_prefix_kernel + decode_split_kernel + decode_merge_kernel"),
                      "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None,
                      "algorithmic_bytes_per_launch": step_bytes, "avg_launch_ms": avg_ms,
                      "peak_source": "%s hbm_gbs" % peaks_src},
-        "gpu_launches": 2 * args.steps,
+        # split + merge, after a prefix kernel when the lengths live on the device
+        "gpu_launches": (2 if sl is None else 3) * args.steps,
         "clocks": clk,
     }
     if e2e:

@@ -57,6 +57,7 @@ constexpr int DEC_CONSUMERS = 8;                     // warps that compute
 constexpr int DEC_THREADS = 32 * (DEC_CONSUMERS + 1);  // + one TMA producer warp
 constexpr int DEC_TILE = 16 * DEC_CONSUMERS;         // keys per TMA tile, 16 per warp
 constexpr int DEC_GMAX = 16;                         // largest Hq / Hkv (MMA rows)
+constexpr int DEC_MERGE_REGS = 8;                    // partials a merge holds in registers
 
 template <int D>
 struct DecodeLayout {
@@ -466,9 +467,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
 
 // Merge the partials of one (sequence, query head): grid B * Hq, D threads
 // (one output column each).  The pair's partials sit in the slots pair + c
-// of the CTAs c whose ranges overlap its tiles.  Their weights e^(lse_s -
-// max) go through shared memory D at a time, so that every thread's sum is
-// a run of independent loads.
+// of the CTAs c whose ranges overlap its tiles.  Up to DEC_MERGE_REGS of
+// them are loaded at once into registers (one memory round trip); more go
+// through shared memory D at a time, so that every thread's sum is a run of
+// independent loads.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
   __shared__ float wsh[D];
@@ -477,20 +479,57 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int g = p.group, hk = h / g, hg = h - hk * g;
   const int tid = threadIdx.x;
+  // The pair's slot range.  With every cache full it follows from the
+  // launch parameters alone and is worked out while the split kernel runs;
+  // device-side lengths need the prefix kernel's offsets first.
+  int nt = 0, c0 = 0, c1 = -1;
+  long long T = 0;
+  auto slot_range = [&]() {
+    nt = dec_ntiles(p, b);
+    if (nt == 0) return;
+    T = dec_total(p);
+    const long long off = (long long)p.Hkv * dec_boff(p, b) + (long long)hk * nt;
+    c0 = dec_cta_of(off, T, p.grid);
+    c1 = dec_cta_of(off + nt - 1, T, p.grid);
+  };
+  if (p.seqlens == nullptr) slot_range();
   griddep_wait();   // the split kernel's partials (and, before it, the offsets)
-  const int nt = dec_ntiles(p, b);
+  if (p.seqlens != nullptr) slot_range();
   float acc = 0.f, wsum = 0.f, M = -INFINITY;
   if (nt > 0) {
-    const long long T = dec_total(p);
-    const long long off = (long long)p.Hkv * dec_boff(p, b) + (long long)hk * nt;
-    const int c0 = dec_cta_of(off, T, p.grid), c1 = dec_cta_of(off + nt - 1, T, p.grid);
     const int ns = c1 - c0 + 1;
     const long long s0 = (long long)b * p.Hkv + hk + c0;   // first slot
-    // a CTA between c0 and c1 with an empty range (more CTAs than tiles)
-    // wrote no partial: it is skipped
+    // a CTA between c0 and c1 with an empty range wrote no partial: it is
+    // skipped.  Empty ranges exist only with more CTAs than tiles.
+    const bool all_ranges = T >= p.grid;
     auto has_range = [&](int c) {
-      return dec_range_start(c, T, p.grid) < dec_range_start(c + 1, T, p.grid);
+      return all_ranges || dec_range_start(c, T, p.grid) < dec_range_start(c + 1, T, p.grid);
     };
+    if (ns <= DEC_MERGE_REGS) {
+      // the usual case: every partial of this thread's column and every
+      // partial LSE loaded at once, then weighed in registers
+      float l[DEC_MERGE_REGS], v[DEC_MERGE_REGS];
+#pragma unroll
+      for (int k = 0; k < DEC_MERGE_REGS; ++k) {
+        l[k] = -INFINITY;
+        v[k] = 0.f;
+        if (k < ns && has_range(c0 + k)) {
+          l[k] = p.lse_part[(s0 + k) * g + hg];
+          v[k] = p.o_part[((s0 + k) * g + hg) * D + tid];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < DEC_MERGE_REGS; ++k) M = fmaxf(M, l[k]);
+#pragma unroll
+      for (int k = 0; k < DEC_MERGE_REGS; ++k) {
+        const float w = (l[k] == -INFINITY) ? 0.f : expf(l[k] - M);
+        wsum += w;
+        acc = fmaf(w, v[k], acc);
+      }
+      p.o[(long long)bh * D + tid] = __float2bfloat16_rn(acc / wsum);
+      if (tid == 0) p.lse[bh] = M + logf(wsum);
+      return;
+    }
     float mx = -INFINITY;
     for (int s = tid; s < ns; s += D)
       if (has_range(c0 + s)) mx = fmaxf(mx, p.lse_part[(s0 + s) * g + hg]);

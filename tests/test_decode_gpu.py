@@ -92,6 +92,8 @@ def _custom(B, Hq, Hkv, Lmax, d, lengths=None, seed=0):
     (64, 4, 4, 100, 128, None),                 # one tile per pair: no partials at all
     (1, 16, 1, 40000, 128, None),               # one pair over every CTA: 148 partials
     (1, 1, 1, 20000, 64, None),                 # a single query head over every CTA
+    (1, 4, 1, 512, 64, [256]),                  # 3 slots, the middle CTA empty
+    (2, 8, 2, 512, 128, [300, 0]),              # 6 slots with empty CTAs, an empty sequence
 ])
 def test_decode_matches_oracle(B, Hq, Hkv, Lmax, d, lengths):
     inp = _custom(B, Hq, Hkv, Lmax, d, lengths, seed=Lmax)
