@@ -42,6 +42,7 @@
 // bulk asynchronous reductions was slower -- the reductions from one issuing
 // thread proceed nearly one after another.)
 #pragma once
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 
@@ -114,8 +115,10 @@ __device__ __forceinline__ long stat_index(const BwdParams& p, int b, int h, int
 // ============================================================================
 // K2: D = rowsum(dO o O) and zeroing of the dQ accumulator
 // ============================================================================
+// Grid-stride; 8 blocks of 256 threads fit on an SM at the 32 registers the
+// launch bound asks for, so the launch (8 blocks per SM) is a single wave.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long tokens) {
+__global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long tokens) {
   // zero the accumulator
   {
     float4* acc = reinterpret_cast<float4*>(p.dq_acc);
@@ -169,45 +172,64 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p, long to
 // ============================================================================
 // K4: dQ = scale * accumulator -> bf16 [token][head][d]
 // ============================================================================
-// grid: (query tiles of the longest sequence, Hq, B); 256 threads; each block
-// turns one 128-row tile (two halves of 64 rows) back into token-major bf16.
+// Persistent: a few blocks per SM stride over the (query tile, head,
+// sequence) items, item = (b * Hq + h) * nq + i; 256 threads turn one
+// 128-row tile (two halves of 64 rows) back into token-major bf16.  Each
+// thread issues all its loads of a half before its shared-memory stores.
+// The staging rows are D + 4 floats apart, so the float4 stores (eight
+// consecutive rows per phase) hit eight different 16-byte bank groups, and
+// so do the two float4 loads of a row's 8-column chunk when every other
+// group of four chunks takes its two halves in swapped order.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long items, int nq) {
   constexpr int RH = 64;                       // rows per half
-  __shared__ float tile[RH][D + 4];
-  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  int seq_start = 0, len = p.N;
-  if (p.cu_seqlens != nullptr) {
-    seq_start = p.cu_seqlens[b];
-    len = p.cu_seqlens[b + 1] - seq_start;
-  }
-  if (128 * i >= len) return;
-  const long tok0 = ((p.cu_seqlens != nullptr) ? (long)seq_start : (long)b * p.N) + 128 * i;
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + acc_tile_offset<D>(p, h, tile_base(p, b) + i));
-  for (int half = 0; half < 2; ++half) {
-    const int r0 = half * RH;
-    if (128 * i + r0 >= len) break;
-    for (int idx = threadIdx.x; idx < (D / 4) * RH; idx += blockDim.x) {
-      const int cg = idx / RH, rr = idx % RH;
-      const float4 v = src[cg * 128 + r0 + rr];
-      tile[rr][4 * cg + 0] = v.x;
-      tile[rr][4 * cg + 1] = v.y;
-      tile[rr][4 * cg + 2] = v.z;
-      tile[rr][4 * cg + 3] = v.w;
+  constexpr int LD = (D / 4) * RH / 256;       // float4 loads per thread and half
+  __shared__ __align__(16) float tile[RH][D + 4];
+  const int tid = threadIdx.x;
+  for (long it = blockIdx.x; it < items; it += gridDim.x) {
+    const int i = (int)(it % nq);
+    const long bh = it / nq;
+    const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+    int seq_start = 0, len = p.N;
+    if (p.cu_seqlens != nullptr) {
+      seq_start = p.cu_seqlens[b];
+      len = p.cu_seqlens[b + 1] - seq_start;
     }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < RH * (D / 8); idx += blockDim.x) {
-      const int rr = idx / (D / 8), ch = idx % (D / 8);
-      if (128 * i + r0 + rr >= len) continue;
-      const float* f = &tile[rr][8 * ch];
-      uint4 w;
-      w.x = pack_bf16(f[0] * p.scale, f[1] * p.scale);
-      w.y = pack_bf16(f[2] * p.scale, f[3] * p.scale);
-      w.z = pack_bf16(f[4] * p.scale, f[5] * p.scale);
-      w.w = pack_bf16(f[6] * p.scale, f[7] * p.scale);
-      *reinterpret_cast<uint4*>(p.dq + ((tok0 + r0 + rr) * p.Hq + h) * D + 8 * ch) = w;
+    if (128 * i >= len) continue;   // the same for the whole block
+    const long tok0 = ((p.cu_seqlens != nullptr) ? (long)seq_start : (long)b * p.N) + 128 * i;
+    const float4* src =
+        reinterpret_cast<const float4*>(p.dq_acc + acc_tile_offset<D>(p, h, tile_base(p, b) + i));
+    for (int half = 0; half < 2; ++half) {
+      const int r0 = half * RH;
+      if (128 * i + r0 >= len) break;
+      float4 v[LD];
+#pragma unroll
+      for (int k = 0; k < LD; ++k) {
+        const int idx = tid + 256 * k;
+        v[k] = src[(idx / RH) * 128 + r0 + idx % RH];
+      }
+#pragma unroll
+      for (int k = 0; k < LD; ++k) {
+        const int idx = tid + 256 * k;
+        *reinterpret_cast<float4*>(&tile[idx % RH][4 * (idx / RH)]) = v[k];
+      }
+      __syncthreads();
+      for (int idx = tid; idx < RH * (D / 8); idx += 256) {
+        const int rr = idx / (D / 8), ch = idx % (D / 8);
+        if (128 * i + r0 + rr >= len) continue;
+        const int sw = (ch >> 2) & 1;
+        const float4 x = *reinterpret_cast<const float4*>(&tile[rr][8 * ch + 4 * sw]);
+        const float4 y = *reinterpret_cast<const float4*>(&tile[rr][8 * ch + 4 - 4 * sw]);
+        const float4 lo = sw ? y : x, hi = sw ? x : y;
+        uint4 w;
+        w.x = pack_bf16(lo.x * p.scale, lo.y * p.scale);
+        w.y = pack_bf16(lo.z * p.scale, lo.w * p.scale);
+        w.z = pack_bf16(hi.x * p.scale, hi.y * p.scale);
+        w.w = pack_bf16(hi.z * p.scale, hi.w * p.scale);
+        *reinterpret_cast<uint4*>(p.dq + ((tok0 + r0 + rr) * p.Hq + h) * D + 8 * ch) = w;
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
 }
 
@@ -758,8 +780,12 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
                          const CUtensorMap& mdo, const BwdParams& p, cudaStream_t stream,
                          cudaEvent_t ev_begin, cudaEvent_t ev_end) {
   const long tokens = (p.cu_seqlens != nullptr) ? (long)p.total : (long)p.B * p.N;
-  bwd_pre_kernel<D><<<148 * 8, 256, 0, stream>>>(p, tokens);
-  cudaError_t e = cudaGetLastError();
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  bwd_pre_kernel<D><<<sms * 8, 256, 0, stream>>>(p, tokens);
+  e = cudaGetLastError();
   if (e != cudaSuccess) {
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: pre kernel launch\n");
     return e;
@@ -780,8 +806,16 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: main kernel launch\n");
     return e;
   }
-  dim3 g2((unsigned)((p.N + 127) / 128), (unsigned)p.Hq, (unsigned)p.B);
-  bwd_dq_kernel<D><<<g2, 256, 0, stream>>>(p);
+  const int nq = (p.N + 127) / 128;
+  const long items = (long)nq * p.Hq * p.B;
+  static int dq_blocks_per_sm = 0;   // per instantiation; the same on every B200
+  if (dq_blocks_per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&dq_blocks_per_sm, bwd_dq_kernel<D>, 256, 0);
+    if (e != cudaSuccess) return e;
+    if (dq_blocks_per_sm < 1) dq_blocks_per_sm = 1;
+  }
+  const long g2 = std::min<long>(items, (long)sms * dq_blocks_per_sm);
+  bwd_dq_kernel<D><<<(unsigned)g2, 256, 0, stream>>>(p, items, nq);
   return cudaGetLastError();
 }
 
