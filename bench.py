@@ -168,6 +168,25 @@ def cpu_sample(w, heads, nthreads):
     return dt, heads * per_head * 3.5
 
 
+def cpu_model():
+    """The host CPU's model name (first processor in /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_per_core(w):
+    """TFLOP/s of the fp64 oracle on one (batch, query head) problem with one
+    thread: the per-core figure beside the all-cores baseline."""
+    dt, f = cpu_sample(w, 1, 1)
+    return f / dt / 1e12
+
+
 def run_reference(args, w):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -192,7 +211,8 @@ def run_reference(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, **w.describe()},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample, "cpu_model": cpu_model(),
+                             "per_core_value": cpu_per_core(w)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -398,7 +418,10 @@ def run_b200(args, w):
             "value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "seconds": dt,
             "sample": "%d (batch, query head) problems of the workload (N=%d, d=%d, causal=%s), "
-                      "fp64 oracle forward + backward" % (heads, w.N, w.d, w.causal)}
+                      "fp64 oracle forward + backward" % (heads, w.N, w.d, w.causal),
+            "cpu_model": cpu_model(),
+            # one problem on one thread
+            "per_core_value": cpu_per_core(w)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -71,4 +71,5 @@ def test_reference_arm_rank0_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert "cpu_model" in line["cpu_baseline"] and line["cpu_baseline"]["per_core_value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
