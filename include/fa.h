@@ -189,7 +189,12 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  *                      fa_decode_workspace_size() bytes, 256-byte aligned,
  *                      for the per-chunk partial results
  * The cache is cut into chunks processed in parallel and merged exactly
- * (lse = ln sum_s e^(lse_s), o = sum_s e^(lse_s - lse) o_s).  d must be 64
+ * (lse = ln sum_s e^(lse_s), o = sum_s e^(lse_s - lse) o_s): a split
+ * kernel and a merge kernel, after a one-block prefix kernel when
+ * cache_seqlens is given.  The split and merge kernels are programmatic
+ * dependent launches; each waits for the kernel before it on the stream
+ * before touching memory, and the last one lets no later kernel start
+ * early, so the call keeps ordinary stream order for the caller's work.  d must be 64
  * or 128 and Hq / Hkv at most 16 (FA_ERR_UNSUPPORTED otherwise); B and Hkv
  * at most 65535.  Same pointer, device, error and stream rules as fa_fwd.
  */
