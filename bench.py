@@ -39,8 +39,11 @@ DECODE_METRIC = "decode attention over a KV cache: GB/s of K/V cache read (bf16,
 SPARSE_METRIC = ("block-sparse attention fwd+bwd TFLOP/s on the allowed (query, key) pairs "
                  "(bf16, 1×B200) and % of dense BF16 tensor peak")
 L2_FLUSH_BYTES = 256 << 20
-DEFAULT_WORKLOAD = "gqa_causal_b2_hq32_hkv8_n4096_d128"
+DEFAULT_WORKLOAD = "long_causal_b1_h16_n65536_d128_x8row"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# SM clock at which the measured sustained bf16 figure was taken, when the
+# peaks file does not record it (1342 MHz under the 1000 W cap)
+SUSTAINED_PEAK_MHZ = 1342.0
 
 
 def load_peaks():
@@ -141,31 +144,63 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle
-def cpu_sample(w, heads, nthreads):
-    """fp64 oracle forward + backward on `heads` (batch, query head) problems of
-    workload w (full sequence length, its causal flag and d), packed as a batch
-    of independent single-head problems.  Returns (seconds, flops)."""
+_INPUTS = {}
+
+
+def _inputs(w):
+    """The workload's seeded inputs, drawn once per process."""
+    from exact_io_aware_67_b200 import workloads
+    key = (w.name, w.seed)
+    if key not in _INPUTS:
+        _INPUTS.clear()
+        _INPUTS[key] = workloads.generate(w)
+    return _INPUTS[key]
+
+
+def cpu_rows_sample(w, nrows, nthreads, seed=0, problems=2):
+    """fp64 oracle on `nrows` query rows of workload w at seeded positions,
+    split over `problems` (batch, query head) problems (the first and the
+    last, then evenly spaced ones): O, LSE, D and dQ of each row (the
+    oracle's row sampler; those outputs depend on the row alone).  Each
+    problem's rows go to the oracle in one call, so its threads share them.
+    Returns (seconds, flops, description).  FLOPs count the work the
+    definition does for those rows: 2 d per allowed key for each of S,
+    O = P V, dP and dQ, i.e. 8 d per allowed key."""
     import numpy as np
     import oracle
-    from exact_io_aware_67_b200 import workloads
-    inp = workloads.generate(w)
+    inp = _inputs(w)
     g = w.Hq // w.Hkv
-    qs, ks, vs, ds = [], [], [], []
-    for u in range(heads):
+    rng = np.random.default_rng(seed)
+    total = w.B * w.Hq
+    npb = max(1, min(problems, total))
+    picks = sorted(set(int(round(x)) for x in np.linspace(0, total - 1, npb)))
+    secs, flops, used = 0.0, 0.0, 0
+    for n, u in enumerate(picks):
         b, h = divmod(u, w.Hq)
-        b %= w.B
-        qs.append(inp.q[b, :, h].float().numpy())
-        ks.append(inp.k[b, :, h // g].float().numpy())
-        vs.append(inp.v[b, :, h // g].float().numpy())
-        ds.append(inp.dout[b, :, h].float().numpy())
-    st = lambda a: np.stack(a)[:, :, None, :].astype(np.float64)
-    q, k, v, do = st(qs), st(ks), st(vs), st(ds)
-    t0 = time.perf_counter()
-    oracle.attention_fwd(q, k, v, w.scale, w.causal, nthreads=nthreads)
-    oracle.attention_bwd(q, k, v, do, w.scale, w.causal, nthreads=nthreads)
-    dt = time.perf_counter() - t0
-    per_head = 4.0 * w.N * w.N * w.d * (0.5 if w.causal else 1.0)
-    return dt, heads * per_head * 3.5
+        take = nrows // len(picks) + (1 if n < nrows % len(picks) else 0)
+        if inp.cu_seqlens is None:
+            sl = lambda t, hh: t[b, :, hh]
+            L = w.N
+        else:
+            st = int(inp.cu_seqlens[b])
+            L = int(inp.cu_seqlens[b + 1]) - st
+            sl = lambda t, hh: t[st:st + L, hh]
+        if L == 0 or take == 0:
+            continue
+        one = lambda t, hh: sl(t, hh)[None, :, None, :].float().numpy().astype(np.float64)
+        q, k, v, do = one(inp.q, h), one(inp.k, h // g), one(inp.v, h // g), one(inp.dout, h)
+        rows = rng.integers(0, L, take)
+        sel = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, do, sel, w.scale, w.causal, nthreads=nthreads)
+        secs += time.perf_counter() - t0
+        keys = (rows + 1) if w.causal else np.full_like(rows, L)
+        flops += 8.0 * w.d * float(keys.sum())
+        used += take
+    desc = ("%d query rows of %s at seeded positions in %d (batch, query head) problems: fp64 "
+            "oracle O, LSE, D and dQ of each row; FLOPs = 8 d per allowed key" %
+            (used, w.name, len(picks)))
+    return secs, flops, desc
 
 
 def cpu_model():
@@ -180,11 +215,20 @@ def cpu_model():
     return None
 
 
+def rows_for_seconds(w, seconds, nthreads):
+    """Rows that take the oracle about `seconds` on `nthreads` threads,
+    calibrated on a short probe of the same workload."""
+    probe = max(64, nthreads * 16)
+    dt, _, _ = cpu_rows_sample(w, probe, nthreads, seed=12345)
+    rate = probe / max(dt, 1e-6)
+    return max(probe, int(rate * seconds))
+
+
 def cpu_per_core(w):
-    """TFLOP/s of the fp64 oracle on one (batch, query head) problem with one
-    thread: the per-core figure beside the all-cores baseline."""
-    dt, f = cpu_sample(w, 1, 1)
-    return f / dt / 1e12
+    """TFLOP/s of the oracle's row sampler on one thread (a few rows of the
+    same workload): the per-core figure beside the all-cores one."""
+    dt, f, _ = cpu_rows_sample(w, 8, 1, seed=777, problems=1)
+    return f / max(dt, 1e-9) / 1e12
 
 
 def run_reference(args, w):
@@ -192,31 +236,59 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     cores = len(os.sched_getaffinity(0))
-    heads = max(1, min(cores, 16, w.B * w.Hq))
-    for _ in range(args.warmup):
-        cpu_sample(w, heads, cores)
-    times, flops = [], 0.0
-    for _ in range(args.steps):
-        dt, f = cpu_sample(w, heads, cores)
+    # each step is a bounded sample (about 3 s of oracle time), so that the
+    # whole --steps/--warmup run stays within a few minutes
+    nrows = rows_for_seconds(w, 3.0, cores)
+    for it in range(args.warmup):
+        cpu_rows_sample(w, nrows, cores, seed=1000 + it)
+    times, flops, desc = [], [], ""
+    for it in range(args.steps):
+        dt, f, desc = cpu_rows_sample(w, nrows, cores, seed=it)
         times.append(dt)
-        flops = f
+        flops.append(f)
     tot = sum(times)
-    value = flops * len(times) / tot / 1e12
-    sample = ("%d (batch, query head) problems of %s per step (N=%d, d=%d, causal=%s), "
-              "fp64 three-pass oracle forward + analytic backward" %
-              (heads, w.name, w.N, w.d, w.causal))
+    value = sum(flops) / tot / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, **w.describe()},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
-                             "kind": "oracle", "sample": sample, "cpu_model": cpu_model(),
-                             "per_core_value": cpu_per_core(w)},
+                             "kind": "oracle", "sample": "per step: " + desc,
+                             "cpu_model": cpu_model(), "per_core_value": cpu_per_core(w)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def peak_for_clock(peaks, clk):
+    """The dense bf16 peak that applies to a run at the clocks it was sampled
+    at: the measured sustained cuBLAS figure scaled from the SM clock it was
+    measured at to this run's median SM clock, capped at the burst figure
+    (the cap applies whenever the run held its clock).  Returns (peak,
+    source note)."""
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    sus_mhz = None
+    for key, val in peaks.items():
+        kl = key.lower()
+        if "sustained" in kl and ("mhz" in kl or "clock" in kl):
+            try:
+                sus_mhz = float(val)
+                break
+            except (TypeError, ValueError):
+                continue
+    if sus_mhz is None:
+        sus_mhz = SUSTAINED_PEAK_MHZ
+    mhz = clk.get("sm_mhz")
+    if not mhz:
+        return burst, "bf16_tflops (burst; no clock samples)"
+    scaled = sus * float(mhz) / sus_mhz
+    if scaled >= burst:
+        return burst, "bf16_tflops (burst; clock-scaled sustained figure %.0f is higher)" % scaled
+    return scaled, ("bf16_tflops_sustained %.1f at %.0f MHz scaled to the run's median %.0f MHz"
+                    % (sus, sus_mhz, mhz))
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -374,15 +446,8 @@ def run_b200(args, w):
     fwd_tf = fwd_f / (fwd_avg / 1e3) / 1e12
     bwd_tf = bwd_f / (bwd_avg / 1e3) / 1e12
     bwd_all_tf = bwd_f / (sum(bwd_all_ms) / len(bwd_all_ms) / 1e3) / 1e12
-    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak, peak_kind = peak_for_clock(peaks, clk)
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # The measured sustained figure was taken at the clocks cuBLAS settles to
-    # under the power cap; use it only if this run's clocks were held down
-    # too (median SM clock well below max), else the burst figure.
-    smhz, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
-    throttled = bool(smhz and smax and smhz < 0.9 * smax)
-    peak = peak_sus if throttled else peak_burst
-    peak_kind = "bf16_tflops_sustained" if throttled else "bf16_tflops (burst)"
     # dominant kernel: the one with the larger share of the step
     if bwd_avg >= fwd_avg:
         dom, dom_ms, dom_f = "bwd_main_kernel", bwd_avg, bwd_f
@@ -407,7 +472,7 @@ def run_b200(args, w):
         "peak_tflops": peak, "peak_source": "%s %s" % (peaks_src, peak_kind),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak,
-                     "frac_of_sustained_peak": achieved / peak_sus,
+                     "frac_of_burst_peak": achieved / peak_burst,
                      "traffic": traffic,
                      "algorithmic_flops_per_launch": dom_f, "avg_launch_ms": dom_ms},
         "gpu_launches": 4 * args.steps,
@@ -419,16 +484,13 @@ def run_b200(args, w):
                        "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": e2e_max / args.steps}
     if not args.no_cpu_baseline and ws == 1:
+        # a bounded sample of the same workload: about 15 s of oracle time
         cores = len(os.sched_getaffinity(0))
-        heads = max(1, min(cores, 16, w.B * w.Hq))
-        dt, f = cpu_sample(w, heads, cores)
+        nrows = rows_for_seconds(w, 15.0, cores)
+        dt, f, desc = cpu_rows_sample(w, nrows, cores)
         line["cpu_baseline"] = {
             "value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "seconds": dt,
-            "sample": "%d (batch, query head) problems of the workload (N=%d, d=%d, causal=%s), "
-                      "fp64 oracle forward + backward" % (heads, w.N, w.d, w.causal),
-            "cpu_model": cpu_model(),
-            # one problem on one thread
+            "seconds": dt, "sample": desc, "cpu_model": cpu_model(),
             "per_core_value": cpu_per_core(w)}
     print(json.dumps(line), flush=True)
     return 0
@@ -534,7 +596,7 @@ def run_blocksparse(args, bw):
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
     peaks, src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak, peak_kind = peak_for_clock(peaks, clk)
     fwd_tf = fwd_f / (fwd_ms / 1e3) / 1e12
     bwd_tf = bwd_f / (bwd_ms / 1e3) / 1e12
     dom, dom_ms, dom_f = (("bwd_main_kernel", bwd_ms, bwd_f) if bwd_ms >= fwd_ms
@@ -553,7 +615,7 @@ def run_blocksparse(args, bw):
                          "achieved": dom_f / (dom_ms / 1e3) / 1e12, "peak": peak,
                          "unit": "TFLOP/s", "frac": dom_f / (dom_ms / 1e3) / 1e12 / peak,
                          "traffic": None, "algorithmic_flops_per_launch": dom_f,
-                         "avg_launch_ms": dom_ms, "peak_source": "%s bf16_tflops (burst)" % src},
+                         "avg_launch_ms": dom_ms, "peak_source": "%s %s" % (src, peak_kind)},
             "gpu_launches": 4 * args.steps, "clocks": clk}
     print(json.dumps(line), flush=True)
     return 0
@@ -756,8 +818,8 @@ def run_decode(args, w, impl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=600)
-    ap.add_argument("--warmup", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -1,7 +1,8 @@
 // fa_api.cu -- host side of libfa.so: argument validation, TMA descriptor
 // encoding, launch configuration, and the C entry points declared in
-// include/fa.h.  The library allocates no device memory and never
-// synchronises the caller's stream.
+// include/fa.h.  The library allocates no device memory (the one exception
+// is the fixed scratch array behind fa_bwd_noalloc, a file-scope device
+// variable) and never synchronises the caller's stream.
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -160,14 +161,6 @@ void* scratch_on_current_device() {
   }
   return ptr;
 }
-
-}  // namespace
-
-extern "C" {
-
-}  // extern "C"
-
-namespace {
 
 // Block mask of the block-sparse entry points: bytes [*][*][nt][nt] with
 // nt = ceil(N / 128), strides (in elements) per sequence and per kv head.

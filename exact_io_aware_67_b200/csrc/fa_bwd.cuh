@@ -43,6 +43,7 @@
 // thread proceed nearly one after another.)
 #pragma once
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstdlib>
 
@@ -808,11 +809,16 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   }
   const int nq = (p.N + 127) / 128;
   const long items = (long)nq * p.Hq * p.B;
-  static int dq_blocks_per_sm = 0;   // per instantiation; the same on every B200
+  // resident blocks per SM of the convert kernel: per instantiation, the same
+  // on every B200; callers on several host threads may race to fill it, so
+  // it is an atomic (relaxed: any thread's answer is the same number)
+  static std::atomic<int> dq_blocks_cache{0};
+  int dq_blocks_per_sm = dq_blocks_cache.load(std::memory_order_relaxed);
   if (dq_blocks_per_sm == 0) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&dq_blocks_per_sm, bwd_dq_kernel<D>, 256, 0);
     if (e != cudaSuccess) return e;
     if (dq_blocks_per_sm < 1) dq_blocks_per_sm = 1;
+    dq_blocks_cache.store(dq_blocks_per_sm, std::memory_order_relaxed);
   }
   const long g2 = std::min<long>(items, (long)sms * dq_blocks_per_sm);
   bwd_dq_kernel<D><<<(unsigned)g2, 256, 0, stream>>>(p, items, nq);

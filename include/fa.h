@@ -38,8 +38,14 @@
  *   stream       : CUDA stream the kernels are enqueued on
  *
  * Ownership: the caller allocates every buffer (inputs, outputs, and the
- * backward workspace).  The library allocates no device memory, keeps no
- * per-call state, and never synchronises the stream.  All pointers are
+ * backward workspace).  The library allocates no device memory at call time
+ * and never synchronises the stream.  Its only device-resident state is the
+ * error word below and one exception, described at fa_bwd_noalloc(): a fixed
+ * FA_BWD_NOALLOC_SCRATCH_BYTES array that every GPU loading the library
+ * holds until exit, whose device address is cached per device and whose
+ * contents persist from call to call (overlapping fa_bwd_noalloc calls race
+ * on it).  Host-side state is limited to settings (wait limit, profiling
+ * events), cached driver entry points and that per-device address.  All pointers are
  * device pointers on one device and must be 16-byte aligned.  The kernels
  * run on the device that owns q: if it is not the calling thread's current
  * device, the call makes it current (this also gives a thread that has not
