@@ -312,6 +312,7 @@ def run_b200(args, w):
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
     maxlen = (max(lengths) if lengths else w.N) if cu is not None else None
     o = torch.empty_like(q)
+    o_lo = torch.empty_like(q)      # O's rounding residual, read back by the backward
     lse = torch.empty((w.B, w.Hq, w.N) if cu is None else (w.Hq, q.shape[0]),
                       dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -322,9 +323,9 @@ def run_b200(args, w):
     stream = torch.cuda.current_stream()
 
     def step():
-        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse)
+        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse, o_lo=o_lo)
         ops.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, cu, maxlen,
-                          workspace=ws_buf, dq=dq, dk=dk, dv=dv)
+                          workspace=ws_buf, dq=dq, dk=dk, dv=dv, o_lo=o_lo)
 
     ops.fa_clear_device_error()
     for _ in range(args.warmup):
@@ -351,11 +352,11 @@ def run_b200(args, w):
     t_begin.record(stream)
     for s in range(args.steps):
         ops.fa_set_profile_events(ev[s][0], ev[s][1])
-        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse)
+        ops.attention_fwd(q, k, v, w.scale, w.causal, cu, maxlen, out=o, lse=lse, o_lo=o_lo)
         ops.fa_set_profile_events(ev[s][2], ev[s][3])
         ev[s][4].record(stream)
         ops.attention_bwd(q, k, v, o, lse, do, w.scale, w.causal, cu, maxlen,
-                          workspace=ws_buf, dq=dq, dk=dk, dv=dv)
+                          workspace=ws_buf, dq=dq, dk=dk, dv=dv, o_lo=o_lo)
         ev[s][5].record(stream)
     ops.fa_set_profile_events(None, None)
     t_end.record(stream)
@@ -385,6 +386,7 @@ def run_b200(args, w):
         din = [[q, k, v, do], [torch.empty_like(t) for t in (q, k, v, do)]]
         dout_ = [[o, dq, dk, dv], [torch.empty_like(t) for t in (o, dq, dk, dv)]]
         lses = [lse, torch.empty_like(lse)]
+        olos = [o_lo, torch.empty_like(o_lo)]
         wss = [ws_buf, torch.empty_like(ws_buf)]
         h2d = sum(t.numel() * t.element_size() for t in hq)
         d2h = sum(t.numel() * t.element_size() for t in hout[0])
@@ -406,9 +408,10 @@ def run_b200(args, w):
                 ev_in[x].record(s_in)
             stream.wait_event(ev_in[x])
             stream.wait_event(ev_out[x])             # step it-2's results downloaded
-            ops.attention_fwd(qq, kk, vv, w.scale, w.causal, cu, maxlen, out=oo, lse=lses[x])
+            ops.attention_fwd(qq, kk, vv, w.scale, w.causal, cu, maxlen, out=oo, lse=lses[x],
+                              o_lo=olos[x])
             ops.attention_bwd(qq, kk, vv, oo, lses[x], dd, w.scale, w.causal, cu, maxlen,
-                              workspace=wss[x], dq=gq, dk=gk, dv=gv)
+                              workspace=wss[x], dq=gq, dk=gk, dv=gv, o_lo=olos[x])
             ev_cmp[x].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_cmp[x])
@@ -555,6 +558,7 @@ def run_blocksparse(args, bw):
     bm = torch.from_numpy(mask).cuda()
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
     o = torch.empty_like(q)
+    o_lo = torch.empty_like(q)
     wsb = torch.empty(ops.fa_bwd_workspace_size(w.B, w.Hq, w.N, w.d, w.B * w.N),
                       dtype=torch.uint8, device="cuda")
     fwd_f = flops.blocksparse_fwd_flops(bw, mask)
@@ -564,10 +568,11 @@ def run_blocksparse(args, bw):
     def step(evs=None):
         if evs:
             ops.fa_set_profile_events(evs[0], evs[1])
-        ops.attention_fwd_blockmask(q, k, v, bm, w.scale, w.causal, out=o, lse=lse)
+        ops.attention_fwd_blockmask(q, k, v, bm, w.scale, w.causal, out=o, lse=lse, o_lo=o_lo)
         if evs:
             ops.fa_set_profile_events(evs[2], evs[3])
-        ops.attention_bwd_blockmask(q, k, v, o, lse, do, bm, w.scale, w.causal, workspace=wsb)
+        ops.attention_bwd_blockmask(q, k, v, o, lse, do, bm, w.scale, w.causal, workspace=wsb,
+                                    o_lo=o_lo)
         if evs:
             ops.fa_set_profile_events(None, None)
 

@@ -35,6 +35,18 @@ fa_status cuda_fail(cudaError_t e, const char* site) {
   return FA_ERR_CUDA;
 }
 
+// With FA_DEBUG_VALIDATE set in the environment, every varlen fa_fwd /
+// fa_bwd call first enqueues validate_cu_kernel on its stream.
+bool debug_validate() {
+  static const bool on = std::getenv("FA_DEBUG_VALIDATE") != nullptr;
+  return on;
+}
+
+cudaError_t launch_validate_cu(const int* cu, int B, int N, int total, cudaStream_t stream) {
+  fa::validate_cu_kernel<<<1, 256, 0, stream>>>(cu, B, N, total);
+  return cudaGetLastError();
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
   PFN_cuTensorMapEncodeTiled_v12000 f = fn.load();
@@ -177,16 +189,19 @@ fa_status check_mask(const BlockMask& bm, const void* cu_seqlens, int N) {
   return FA_OK;
 }
 
-fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                   int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
-                   int total_tokens, const BlockMask& bm, cudaStream_t stream) {
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, void* o_lo,
+                   int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                   const int* cu_seqlens, int total_tokens, const BlockMask& bm,
+                   cudaStream_t stream) {
   const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
   bool empty = false;
   fa_status st = check_dims(s, scale, &empty);
   if (st != FA_OK) return st;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(o_lo))
     return FA_ERR_INVALID_ARG;
+  if (o_lo != nullptr && o_lo == o) return FA_ERR_INVALID_ARG;
   st = check_mask(bm, cu_seqlens, N);
   if (st != FA_OK) return st;
   if (empty) return FA_OK;
@@ -201,6 +216,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
   fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_lo = static_cast<__nv_bfloat16*>(o_lo);
   p.lse = lse;
   p.cu_seqlens = cu_seqlens;
   p.B = B;
@@ -218,6 +234,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   p.bm_nt = (N + 127) / 128;
 
   cudaError_t e;
+  if (cu_seqlens != nullptr && debug_validate()) {
+    e = launch_validate_cu(cu_seqlens, B, N, total_tokens, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens validation launch");
+  }
   if (bm.m == nullptr) {
     if (d == 64)
       e = causal ? launch_fwd<64, true>(mq, mk, mv, p, stream)
@@ -239,7 +259,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
 
 fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                   const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                   const void* o_lo, const void* dO, void* dq, void* dk, void* dv, void* workspace,
                    size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
                    int causal, const int* cu_seqlens, int total_tokens, const BlockMask& bm,
                    cudaStream_t stream) {
@@ -248,9 +268,10 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   fa_status st = check_dims(s, scale, &empty);
   if (st != FA_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, o_lo};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if (o_lo != nullptr && o_lo == o) return FA_ERR_INVALID_ARG;
   st = check_mask(bm, cu_seqlens, N);
   if (st != FA_OK) return st;
   if (empty) return FA_OK;
@@ -271,6 +292,7 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   fa::BwdParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.o = static_cast<const __nv_bfloat16*>(o);
+  p.o_lo = static_cast<const __nv_bfloat16*>(o_lo);
   p.dout = static_cast<const __nv_bfloat16*>(dO);
   p.lse = lse;
   p.dq = static_cast<__nv_bfloat16*>(dq);
@@ -291,6 +313,10 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   p.bm_sh = bm.sh;
   p.bm_nt = (N + 127) / 128;
   fa::bwd_carve_workspace(p, workspace, s.tokens(), d);
+  if (cu_seqlens != nullptr && debug_validate()) {
+    const cudaError_t ev = launch_validate_cu(cu_seqlens, B, N, total_tokens, stream);
+    if (ev != cudaSuccess) return cuda_fail(ev, "cu_seqlens validation launch");
+  }
 
   const cudaError_t e =
       fa::launch_bwd(mq, mk, mv, mdo, p, d, causal != 0, stream, t_prof_begin, t_prof_end);
@@ -301,19 +327,19 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
 
 extern "C" {
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                 int Hkv, int N, int d, float scale, int causal, const int* cu_seqlens,
-                 int total_tokens, cudaStream_t stream) {
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, total_tokens,
-                  BlockMask{nullptr, 0, 0}, stream);
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_lo,
+                 int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
+  return fwd_impl(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, causal, cu_seqlens,
+                  total_tokens, BlockMask{nullptr, 0, 0}, stream);
 }
 
-fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                           int Hq, int Hkv, int N, int d, float scale, int causal,
-                           const unsigned char* block_mask, long mask_batch_stride,
+fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse,
+                           void* o_lo, int B, int Hq, int Hkv, int N, int d, float scale,
+                           int causal, const unsigned char* block_mask, long mask_batch_stride,
                            long mask_head_stride, cudaStream_t stream) {
   if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
-  return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, nullptr, B * N,
+  return fwd_impl(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, causal, nullptr, B * N,
                   BlockMask{block_mask, mask_batch_stride, mask_head_stride}, stream);
 }
 
@@ -327,27 +353,29 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
-                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
-                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+                 const void* o_lo, const void* dO, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                 float scale, int causal, const int* cu_seqlens, int total_tokens,
+                 cudaStream_t stream) {
+  return bwd_impl(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
                   scale, causal, cu_seqlens, total_tokens, BlockMask{nullptr, 0, 0}, stream);
 }
 
 fa_status fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
-                           const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                           void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N,
-                           int d, float scale, int causal, const unsigned char* block_mask,
-                           long mask_batch_stride, long mask_head_stride, cudaStream_t stream) {
+                           const float* lse, const void* o_lo, const void* dO, void* dq,
+                           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                           int Hq, int Hkv, int N, int d, float scale, int causal,
+                           const unsigned char* block_mask, long mask_batch_stride,
+                           long mask_head_stride, cudaStream_t stream) {
   if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+  return bwd_impl(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
                   scale, causal, nullptr, B * N,
                   BlockMask{block_mask, mask_batch_stride, mask_head_stride}, stream);
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
-                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
-                         int Hq, int Hkv, int N, int d, float scale, int causal,
+                         const float* lse, const void* o_lo, const void* dO, void* dq, void* dk,
+                         void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                          const int* cu_seqlens, int total_tokens, cudaStream_t stream) {
   const Dims s{B, Hq, Hkv, N, d, total_tokens, cu_seqlens != nullptr};
   bool empty = false;
@@ -361,8 +389,8 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (st != FA_OK) return st;
   void* scratch = scratch_on_current_device();
   if (scratch == nullptr) return FA_ERR_CUDA;
-  return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Hq, Hkv,
-                N, d, scale, causal, cu_seqlens, total_tokens, stream);
+  return fa_bwd(q, k, v, o, lse, o_lo, dO, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, Hq,
+                Hkv, N, d, scale, causal, cu_seqlens, total_tokens, stream);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d) {
@@ -450,6 +478,16 @@ fa_status fa_std_softmax(const void* s, void* p, float* lse, int BH, int N, floa
   prm.scale_log2 = scale * 1.4426950408889634f;
   const cudaError_t e = fa::launch_std_softmax(prm, stream);
   return e == cudaSuccess ? FA_OK : cuda_fail(e, "standard softmax launch");
+}
+
+fa_status fa_validate_cu_seqlens(const int* cu_seqlens, int B, int N, int total_tokens,
+                                 cudaStream_t stream) {
+  if (cu_seqlens == nullptr || B < 0 || N < 1 || total_tokens < 0) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  const fa_status st = bind_device_of(cu_seqlens);
+  if (st != FA_OK) return st;
+  const cudaError_t e = launch_validate_cu(cu_seqlens, B, N, total_tokens, stream);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e, "cu_seqlens validation launch");
 }
 
 int fa_device_error(void) {

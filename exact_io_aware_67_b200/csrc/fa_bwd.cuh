@@ -10,7 +10,10 @@
 //
 // Three kernels run in stream order:
 //   bwd_pre_kernel     D = rowsum(dO o O) in fp32 and zero the fp32 dQ
-//                      accumulator (HBM-bound, grid-stride).
+//                      accumulator (HBM-bound, grid-stride).  O is the bf16
+//                      output plus, when the forward wrote it, its bf16
+//                      rounding residual: with bf16 O alone the rounding
+//                      error of D reaches dK through -scale P_ij D_i Q_i.
 //   bwd_main_kernel    one CTA per 128-row K/V tile of one (sequence, kv
 //                      head).  It loops over the query heads of its group and
 //                      over the query tiles (only those on or below the
@@ -33,7 +36,9 @@
 // dQ accumulator layout (fp32, tile-major): query tile i of sequence b has
 // its own 128-row block at tile slot  tb(b) + i,  where
 //   tb(b) = b * ceil(N / 128)                 (dense batches)
-//   tb(b) = ceil(cu_seqlens[b] / 128) + b     (variable-length batches),
+//   tb(b) = ceil(start(b) / 128) + b          (variable-length batches; start(b)
+//                                             is cu_seqlens[b] clamped to
+//                                             [0, total]),
 // which never overlaps the next sequence's slots.  Inside a slot the layout
 // is [head][column group of 4][row 0..127][4], so the 32 threads of a warp
 // (32 consecutive rows) add one contiguous 512-byte run per vector atomic.
@@ -55,6 +60,7 @@ namespace fa {
 struct BwdParams {
   const __nv_bfloat16* q;
   const __nv_bfloat16* o;
+  const __nv_bfloat16* o_lo;   // optional bf16 rounding residual of O (nullptr: none)
   const __nv_bfloat16* dout;
   const float* lse;
   __nv_bfloat16* dq;
@@ -63,6 +69,7 @@ struct BwdParams {
   float* dpsum;      // D, same layout as lse
   float* dq_acc;     // fp32 dQ accumulator (layout above)
   long tile_slots;   // tile slots of the accumulator per head
+  int order_chunk;   // (sequence, kv head) pairs per dispatch chunk (causal grid order)
   const int* cu_seqlens;
   int B, Hq, Hkv, N, group, total;
   float scale, scale_log2;
@@ -94,10 +101,13 @@ inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int /*d*/) 
   p.tile_slots = bwd_tile_slots(p.B, p.N, tokens, p.cu_seqlens != nullptr);
 }
 
-// first tile slot of sequence b
+// first tile slot of sequence b (from its clamped start, so that a corrupt
+// cu_seqlens still keeps every slot below tile_slots)
 __device__ __forceinline__ long tile_base(const BwdParams& p, int b) {
-  return (p.cu_seqlens != nullptr) ? (long)((p.cu_seqlens[b] + 127) / 128) + b
-                                   : (long)b * ((p.N + 127) / 128);
+  if (p.cu_seqlens == nullptr) return (long)b * ((p.N + 127) / 128);
+  int start, len;
+  seq_range(p.cu_seqlens, b, p.total, &start, &len);
+  return (long)((start + 127) / 128) + b;
 }
 
 // fp32 offset of (head h, tile slot ts, column group 0, row 0)
@@ -143,14 +153,19 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
     if (row < rows) {
       const uint4 a = *reinterpret_cast<const uint4*>(p.o + row * D + li * 8);
       const uint4 b = *reinterpret_cast<const uint4*>(p.dout + row * D + li * 8);
-      const __nv_bfloat162* ah = reinterpret_cast<const __nv_bfloat162*>(&a);
-      const __nv_bfloat162* bh = reinterpret_cast<const __nv_bfloat162*>(&b);
+      uint4 c = make_uint4(0u, 0u, 0u, 0u);
+      if (p.o_lo != nullptr) c = *reinterpret_cast<const uint4*>(p.o_lo + row * D + li * 8);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+      const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 x = __bfloat1622float2(ah[e]);
-        const float2 y = __bfloat1622float2(bh[e]);
-        s = fmaf(x.x, y.x, s);
-        s = fmaf(x.y, y.y, s);
+        // O = bf16(O) + residual: exact in fp32 (about 16 significant bits)
+        const float2 x = unpack_bf16(av[e]);
+        const float2 xr = unpack_bf16(cv[e]);
+        const float2 y = unpack_bf16(bv[e]);
+        s = fmaf(x.x + xr.x, y.x, s);
+        s = fmaf(x.y + xr.y, y.y, s);
       }
     }
 #pragma unroll
@@ -192,10 +207,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long ite
     const long bh = it / nq;
     const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
     int seq_start = 0, len = p.N;
-    if (p.cu_seqlens != nullptr) {
-      seq_start = p.cu_seqlens[b];
-      len = p.cu_seqlens[b + 1] - seq_start;
-    }
+    if (p.cu_seqlens != nullptr) seq_range(p.cu_seqlens, b, p.total, &seq_start, &len);
     if (128 * i >= len) continue;   // the same for the whole block
     const long tok0 = ((p.cu_seqlens != nullptr) ? (long)seq_start : (long)b * p.N) + 128 * i;
     const float4* src =
@@ -305,22 +317,37 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint8_t* smem = L::SLACK ? align_1024(smem_raw) : smem_raw;
 
   // ---------------------------------------------------------------- work item
-  // Blocks are dispatched roughly in index order.  Causal: the K/V tile
-  // index is slowest, so the longest blocks (tile j has nq - j query tiles)
-  // start first and the short ones fill the tail -- at B=2, Hkv=8, N=4096
-  // this took the main kernel from 737 to 912 TFLOP/s on B200.  Without the
-  // mask every tile of a sequence has the same work, and the tiles of one
-  // (sequence, kv head) stay adjacent so that they share Q and dO in L2.
+  // Blocks are dispatched roughly in index order.  Causal: the (sequence, kv
+  // head) pairs are cut into chunks of order_chunk pairs; within a chunk the
+  // K/V tile index is slowest, so the longest blocks (tile j has nq - j query
+  // tiles) start first and the short ones fill the chunk's tail -- at B=2,
+  // Hkv=8, N=4096 (one chunk) this took the main kernel from 737 to 912
+  // TFLOP/s on B200.  A chunk holds at least four waves of blocks, so the
+  // tails still interleave, while the blocks in flight touch only the chunk's
+  // Q, dO and dQ-accumulator tiles, which then stay in L2 between the blocks
+  // that share them (at N = 65536 the accumulator is four times the L2).
+  // Without the mask every tile of a sequence has the same work, and the
+  // tiles of one (sequence, kv head) stay adjacent to share Q and dO in L2.
   const unsigned nkv_blocks = (unsigned)(p.N + 127) / 128;
   const unsigned bh = (unsigned)p.Hkv * p.B;
-  const unsigned u = CAUSAL ? (blockIdx.x % bh) : (blockIdx.x / nkv_blocks);
-  const int j = (int)(CAUSAL ? blockIdx.x / bh : blockIdx.x % nkv_blocks);
+  unsigned u;
+  int j;
+  if (CAUSAL) {
+    const unsigned chunk = (unsigned)p.order_chunk;
+    const unsigned c = blockIdx.x / (chunk * nkv_blocks);
+    const unsigned r = blockIdx.x - c * chunk * nkv_blocks;
+    const unsigned pairs = min(chunk, bh - c * chunk);
+    u = c * chunk + r % pairs;
+    j = (int)(r / pairs);
+  } else {
+    u = blockIdx.x / nkv_blocks;
+    j = (int)(blockIdx.x % nkv_blocks);
+  }
   const int hk = (int)(u % p.Hkv);
   const int b = (int)(u / p.Hkv);
   int seq_start = 0, len = p.N, bcoord = b;
   if (p.cu_seqlens != nullptr) {
-    seq_start = p.cu_seqlens[b];
-    len = p.cu_seqlens[b + 1] - seq_start;
+    seq_range(p.cu_seqlens, b, p.total, &seq_start, &len);
     bcoord = 0;
   }
   if (128 * j >= len) return;
@@ -471,10 +498,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                       seq_start + 128 * i, bcoord);
       }
       do_issued = n + 1;
-      // statistics of the 128 query rows: LSE * log2(e) and D; rows past the
-      // sequence end get +inf / 0 so that their P and dS vanish.  The stage's
-      // previous readers are done: they finished before dK of iteration n-2,
-      // which released q_empty[s].
+      // statistics of the 128 query rows, negated for the packed elementwise
+      // math: -LSE * log2(e) and -D; rows past the sequence end get -inf / 0
+      // so that their P and dS vanish.  The stage's previous readers are
+      // done: they finished before dK of iteration n-2, which released
+      // q_empty[s].
       float lv[4], dv[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -488,8 +516,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       for (int e = 0; e < 4; ++e) {
         const int r = lane + 32 * e;
         const bool valid = 128 * i + r < len;
-        st[r] = valid ? lv[e] * kLog2e : INFINITY;
-        st[128 + r] = valid ? dv[e] : 0.f;
+        st[r] = valid ? -lv[e] * kLog2e : -INFINITY;
+        st[128 + r] = valid ? -dv[e] : 0.f;
       }
       mbar_arrive(st_full + s);
     }
@@ -674,13 +702,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_ld32(tS + 32, sv + 32);
         tmem_wait_ld32(sv);
         tmem_wait_ld32(sv + 32);
+        // x = s c2 - LSE log2(e) in packed pairs (the stats hold -LSE log2 e)
+        const float2 c22 = make_float2(c2, c2);
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
           const float4 l4 = *reinterpret_cast<const float4*>(st + 64 * wg + 4 * c4);
-          P[4 * c4 + 0] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 0]), c2, -l4.x));
-          P[4 * c4 + 1] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 1]), c2, -l4.y));
-          P[4 * c4 + 2] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 2]), c2, -l4.z));
-          P[4 * c4 + 3] = ex2(fmaf(__uint_as_float(sv[4 * c4 + 3]), c2, -l4.w));
+          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 0]),
+                                               __uint_as_float(sv[4 * c4 + 1])),
+                                   c22, make_float2(l4.x, l4.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 2]),
+                                               __uint_as_float(sv[4 * c4 + 3])),
+                                   c22, make_float2(l4.z, l4.w));
+          P[4 * c4 + 0] = ex2(x01.x);
+          P[4 * c4 + 1] = ex2(x01.y);
+          P[4 * c4 + 2] = ex2(x23.x);
+          P[4 * c4 + 3] = ex2(x23.y);
         }
         // masks (warp-uniform test first): causal diagonal tile -- key row
         // kv_row is masked for query q < kv_row -- and key rows past the end
@@ -712,16 +748,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_wait_ld32(dv);
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
+          // dS = P (dP - D) (the stats hold -D)
           const float4 d4 = *reinterpret_cast<const float4*>(st + 128 + 64 * wg + 32 * hh + 4 * c4);
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-          float ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 32 * hh + 4 * c4 + e;
-            ds[e] = P[c] * (__uint_as_float(dv[4 * c4 + e]) - dd[e]);
-          }
-          dsp[16 * hh + 2 * c4] = pack_bf16(ds[0], ds[1]);
-          dsp[16 * hh + 2 * c4 + 1] = pack_bf16(ds[2], ds[3]);
+          const int c = 32 * hh + 4 * c4;
+          const float2 ds01 = make_float2(P[c] * (__uint_as_float(dv[4 * c4 + 0]) + d4.x),
+                                          P[c + 1] * (__uint_as_float(dv[4 * c4 + 1]) + d4.y));
+          const float2 ds23 = make_float2(P[c + 2] * (__uint_as_float(dv[4 * c4 + 2]) + d4.z),
+                                          P[c + 3] * (__uint_as_float(dv[4 * c4 + 3]) + d4.w));
+          dsp[16 * hh + 2 * c4] = pack_bf16(ds01.x, ds01.y);
+          dsp[16 * hh + 2 * c4 + 1] = pack_bf16(ds23.x, ds23.y);
         }
       }
       // the previous dS tile must have been consumed by its dK and dQ products
@@ -793,6 +828,15 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   }
   auto kern = bwd_main_kernel<D, CAUSAL, SPARSE>;
   const int smem = BwdLayout<D>::ALLOC;
+  // causal dispatch chunks: the fewest (sequence, kv head) pairs whose blocks
+  // make at least four waves (one block per SM)
+  BwdParams pc = p;
+  {
+    const long nkv = (p.N + 127) / 128;
+    const long bh = (long)p.Hkv * p.B;
+    const long want = (4L * sms + nkv - 1) / nkv;
+    pc.order_chunk = (int)std::max(1L, std::min(bh, want));
+  }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) {
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: set smem attribute\n");
@@ -800,7 +844,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   }
   const unsigned grid = (unsigned)((p.N + 127) / 128) * p.Hkv * p.B;
   if (ev_begin != nullptr) cudaEventRecord(ev_begin, stream);
-  kern<<<grid, BWD_THREADS, smem, stream>>>(mq, mk, mv, mdo, p);
+  kern<<<grid, BWD_THREADS, smem, stream>>>(mq, mk, mv, mdo, pc);
   e = cudaGetLastError();
   if (e == cudaSuccess && ev_end != nullptr) e = cudaEventRecord(ev_end, stream);
   if (e != cudaSuccess) {

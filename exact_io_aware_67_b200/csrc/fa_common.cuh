@@ -34,10 +34,16 @@ enum : int {
   ERR_SELFTEST = 0x301,
   ERR_DEC_KV_FULL = 0x401,
   ERR_DEC_KV_EMPTY = 0x402,
+  // cu_seqlens validation (validate_cu_kernel): the lowest failing rule wins
+  ERR_CU_FIRST = 0x501,        // cu[0] != 0
+  ERR_CU_DECREASING = 0x502,   // cu[b + 1] < cu[b]
+  ERR_CU_TOO_LONG = 0x503,     // a sequence longer than N
+  ERR_CU_TOTAL = 0x504,        // cu[B] > total_tokens
 };
 
 struct FwdParams {
   __nv_bfloat16* o;
+  __nv_bfloat16* o_lo;     // optional: O - bf16(O), rounded to bf16 (nullptr: not written)
   float* lse;
   const int* cu_seqlens;   // nullptr for dense inputs
   int B, Hq, Hkv, N, group;
@@ -59,6 +65,44 @@ constexpr int FA_SPARSE_MAX_TILES = 512;
 // Device error word of the library (first error wins; 0 = none).  All
 // kernels live in one translation unit, so one definition serves them all.
 __device__ int g_fa_error = 0;
+
+// Token range [*start, *start + *len) of sequence b of a variable-length
+// batch, clamped to [0, total]: whatever cu_seqlens holds (decreasing,
+// negative, past the caller's allocation), every row a kernel derives from
+// it lies inside the buffers.  The results of such a batch are undefined;
+// validate_cu_kernel reports it.
+__device__ __forceinline__ void seq_range(const int* cu, int b, int total, int* start,
+                                          int* len) {
+  const int s = min(max(cu[b], 0), total);
+  const int e = min(max(cu[b + 1], s), total);
+  *start = s;
+  *len = e - s;
+}
+
+// Checks a cu_seqlens array with one block: cu[0] == 0, non-decreasing,
+// every length at most N, cu[B] <= total.  The lowest failing rule's code
+// goes to the error word (first error wins there).  Reads cu[0..B] only.
+__global__ void __launch_bounds__(256) validate_cu_kernel(const int* cu, int B, int N,
+                                                           int total) {
+  __shared__ int worst;
+  if (threadIdx.x == 0) worst = 0x7fffffff;
+  __syncthreads();
+  int code = 0x7fffffff;
+  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+    const int c = cu[b];
+    if (b == 0 && c != 0) code = min(code, (int)ERR_CU_FIRST);
+    if (b < B) {
+      const int nxt = cu[b + 1];
+      if (nxt < c) code = min(code, (int)ERR_CU_DECREASING);
+      else if ((long)nxt - c > (long)N) code = min(code, (int)ERR_CU_TOO_LONG);
+    } else if (c > total) {
+      code = min(code, (int)ERR_CU_TOTAL);
+    }
+  }
+  atomicMin(&worst, code);
+  __syncthreads();
+  if (threadIdx.x == 0 && worst != 0x7fffffff) atomicCAS(&g_fa_error, 0, worst);
+}
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);

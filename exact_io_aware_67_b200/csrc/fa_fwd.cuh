@@ -76,14 +76,11 @@ static_assert(128 * (2 * FWD_REGS_SOFTMAX + FWD_REGS_CTRL) <= 65536 &&
               "register split");
 constexpr float RESCALE_LOG2 = 8.0f;
 // Pairs out of every 8 column pairs whose exp2 runs on the FMA pipe
-// (ex2_poly) instead of MUFU.  Measured on B200 (forward TFLOP/s, causal
-// H=16 N=16384 d=64): 0 -> 716, 2 -> 651, 3 -> 606, 4 -> 565, and slower at
-// d=128 too: the scalar cubic costs more issue slots than the MUFU time it
-// frees, so 0.  (Taking the exponentials against the running max before the
-// tile's max is known, redoing the rare tile whose max moved, was slower as
-// well: 866 vs 1000 at GQA N=4096 d=128, since S then stays live in registers
-// for the whole pass.)
-constexpr int EXP2_POLY_PAIRS_OF_8 = 0;
+// (ex2_poly2, packed) instead of MUFU.
+#ifndef FA_EXP2_POLY_PAIRS
+#define FA_EXP2_POLY_PAIRS 0
+#endif
+constexpr int EXP2_POLY_PAIRS_OF_8 = FA_EXP2_POLY_PAIRS;
 
 template <int D, bool CAUSAL, bool SPARSE = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
@@ -103,8 +100,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const int b = (int)(blockIdx.x % bh) / p.Hq;
   int seq_start = 0, len = p.N, bcoord = b;
   if (p.cu_seqlens != nullptr) {
-    seq_start = p.cu_seqlens[b];
-    len = p.cu_seqlens[b + 1] - seq_start;
+    seq_range(p.cu_seqlens, b, p.total, &seq_start, &len);
     bcoord = 0;
   }
   const int q0 = qb * 256;
@@ -473,30 +469,27 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       // exp2, the rest MUFU.  P (bf16) goes to this row of the 128B-swizzled
       // K-major P tile: columns 0-63 and 64-127 are two 16 KB regions.
       uint8_t* prow = sP + (L::P_SMEM ? t * 32768 + (r >> 3) * 1024 + (r & 7) * 128 : 0);
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // x = s c2 - m and the row sum in packed pairs (half the issue slots)
+      const float2 c22 = make_float2(c2, c2), nm2 = make_float2(neg_m, neg_m);
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(__uint_as_float(s[32 * cc + 2 * i]), c2, neg_m);
-          const float x1 = fmaf(__uint_as_float(s[32 * cc + 2 * i + 1]), c2, neg_m);
-          float p0, p1;
-          if ((i & 7) >= 8 - EXP2_POLY_PAIRS_OF_8) {
-            p0 = ex2_poly(x0);
-            p1 = ex2_poly(x1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
-          if (i & 1) {
-            l2 += p0;
-            l3 += p1;
-          } else {
-            l0 += p0;
-            l1 += p1;
-          }
-          pk[i] = pack_bf16(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(s[32 * cc + 2 * i]),
+                                             __uint_as_float(s[32 * cc + 2 * i + 1])),
+                                 c22, nm2);
+          float2 pp;
+          if ((i & 7) >= 8 - EXP2_POLY_PAIRS_OF_8)
+            pp = ex2_poly2(x);
+          else
+            pp = make_float2(ex2(x.x), ex2(x.y));
+          if (i & 1)
+            lb = fadd2(lb, pp);
+          else
+            la = fadd2(la, pp);
+          pk[i] = pack_bf16(pp.x, pp.y);
         }
         if constexpr (L::P_SMEM) {
           uint8_t* reg = prow + (cc >> 1) * 16384;
@@ -510,7 +503,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
           tmem_st16(tS + 16 * cc, pk);   // P_t over the S_t columns already read
         }
       }
-      l += (l0 + l1) + (l2 + l3);
+      l += (la.x + la.y) + (lb.x + lb.y);
       if constexpr (L::P_SMEM)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       else
@@ -531,6 +524,9 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         const long tok = (p.cu_seqlens != nullptr) ? (long)seq_start + qrow
                                                     : (long)b * p.N + qrow;
         __nv_bfloat16* orow = p.o + (tok * p.Hq + h) * (long)D;
+        // optional second output: the bf16 rounding residual of O, so that
+        // the backward can form D = rowsum(dO o O) from ~16-bit O
+        __nv_bfloat16* lorow = (p.o_lo != nullptr) ? p.o_lo + (tok * p.Hq + h) * (long)D : nullptr;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -546,6 +542,16 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
               dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            if (lorow != nullptr) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16_residual(__uint_as_float(o[2 * i]) * inv_l,
+                                           __uint_as_float(o[2 * i + 1]) * inv_l, pk[i]);
+              uint4* dlo = reinterpret_cast<uint4*>(lorow + 32 * c);
+#pragma unroll
+              for (int v4 = 0; v4 < 4; ++v4)
+                dlo[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            }
           }
         }
         if (row_ok) {
@@ -561,6 +567,11 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       uint4* dst = reinterpret_cast<uint4*>(p.o + (tok * p.Hq + h) * (long)D);
 #pragma unroll 1
       for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+      if (p.o_lo != nullptr) {
+        uint4* dlo = reinterpret_cast<uint4*>(p.o_lo + (tok * p.Hq + h) * (long)D);
+#pragma unroll 1
+        for (int v4 = 0; v4 < D / 8; ++v4) dlo[v4] = make_uint4(0u, 0u, 0u, 0u);
+      }
       p.lse[((long)b * p.Hq + h) * p.N + qrow] = -INFINITY;
     }
   }

@@ -273,22 +273,60 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 2^7 (used for part of a row's exponentials so
-// that the MUFU unit is not the only source).  Range reduction: n = round(x)
-// via the 1.5 * 2^23 rounding constant, f = x - n in [-1/2, 1/2]; 2^f by a
-// cubic whose coefficients minimise the maximum relative error on [-1/2, 1/2]
-// (Remez exchange, exact_io_aware_67_b200/fit_exp2.py: 7.5e-5); 2^n is added
-// to the exponent field.  x is clamped at -125 so the result stays a normal
-// number; below that the true value (< 2^-125) is far under any bf16 or
-// fp32-sum resolution that matters here.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;            // round(x) lands in t's low mantissa bits
-  const float f = x - (t - 12582912.f);      // f in [-1/2, 1/2]
-  float p = fmaf(f, 5.517166853e-02f, 2.426111251e-01f);
-  p = fmaf(p, f, 6.932609677e-01f);
-  p = fmaf(p, f, 9.999280572e-01f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction computes
+// both lanes, halving the issue slots of elementwise fp32 work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe (packed), for x <= 2^7, so that part of a
+// row's exponentials need not queue on the MUFU unit.  Range reduction:
+// n = round(x) via the 1.5 * 2^23 rounding constant (n lands in t's low
+// mantissa bits), f = x - n in [-1/2, 1/2] (exact: x and n are within a
+// factor of two, or n = 0); 2^f by a cubic whose coefficients minimise the
+// maximum relative error on [-1/2, 1/2] (Remez exchange, written for this
+// library: 7.5e-5, far below bf16's 2^-9); n is added to the exponent field.
+// x is clamped at -125 so that the result stays a normal number; below that
+// the true value (< 2^-125) is far under any bf16 or fp32-sum resolution that
+// matters here, and -inf (a masked score) gives a tiny positive value.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(f, make_float2(5.517166853e-02f, 5.517166853e-02f),
+                   make_float2(2.426111251e-01f, 2.426111251e-01f));
+  p = ffma2(p, f, make_float2(6.932609677e-01f, 6.932609677e-01f));
+  p = ffma2(p, f, make_float2(9.999280572e-01f, 9.999280572e-01f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // max of three
@@ -301,6 +339,21 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The two fp32 values of a packed bf16 pair (exact: bf16 is the top half of
+// an fp32).
+__device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+// The rounding residuals x - bf16(x) of a pair whose bf16 rounding is
+// `packed`, themselves rounded to bf16.  The subtraction is exact in fp32
+// (the residual of rounding an fp32 to fewer mantissa bits is representable),
+// so bf16(O) + residual carries about 16 significant bits of O.
+__device__ __forceinline__ uint32_t pack_bf16_residual(float x0, float x1, uint32_t packed) {
+  const float2 r = unpack_bf16(packed);
+  return pack_bf16(x0 - r.x, x1 - r.y);
 }
 
 }  // namespace fa

@@ -25,7 +25,7 @@ EXPORTED = ["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_error",
             "fa_clear_device_error", "fa_set_wait_limit_ns", "fa_watchdog_selftest",
             "fa_status_string", "fa_last_cuda_error", "fa_set_profile_events",
             "fa_bwd_noalloc", "fa_std_softmax", "fa_decode", "fa_decode_workspace_size",
-            "fa_fwd_blockmask", "fa_bwd_blockmask"]
+            "fa_fwd_blockmask", "fa_bwd_blockmask", "fa_validate_cu_seqlens"]
 
 # capacity of the fixed scratch behind fa_bwd_noalloc (include/fa.h)
 FA_BWD_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -59,17 +59,17 @@ def load(build_if_missing=True):
                            % path)
     lib = ctypes.CDLL(path)
     vp, ip, c_int, c_float = ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_float
-    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp] + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
+    lib.fa_fwd.argtypes = [vp] * 6 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
     lib.fa_fwd.restype = c_int
-    lib.fa_bwd.argtypes = [vp] * 10 + [ctypes.c_size_t] + [c_int] * 5 + \
+    lib.fa_bwd.argtypes = [vp] * 11 + [ctypes.c_size_t] + [c_int] * 5 + \
         [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd.restype = c_int
-    lib.fa_bwd_noalloc.argtypes = [vp] * 9 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
+    lib.fa_bwd_noalloc.argtypes = [vp] * 10 + [c_int] * 5 + [c_float, c_int, vp, c_int, vp]
     lib.fa_bwd_noalloc.restype = c_int
     cl = ctypes.c_long
-    lib.fa_fwd_blockmask.argtypes = [vp] * 5 + [c_int] * 5 + [c_float, c_int, vp, cl, cl, vp]
+    lib.fa_fwd_blockmask.argtypes = [vp] * 6 + [c_int] * 5 + [c_float, c_int, vp, cl, cl, vp]
     lib.fa_fwd_blockmask.restype = c_int
-    lib.fa_bwd_blockmask.argtypes = [vp] * 10 + [ctypes.c_size_t] + [c_int] * 5 + \
+    lib.fa_bwd_blockmask.argtypes = [vp] * 11 + [ctypes.c_size_t] + [c_int] * 5 + \
         [c_float, c_int, vp, cl, cl, vp]
     lib.fa_bwd_blockmask.restype = c_int
     lib.fa_decode.argtypes = [vp] * 6 + [c_int] * 5 + [c_float, vp, ctypes.c_size_t, vp]
@@ -80,6 +80,8 @@ def load(build_if_missing=True):
     lib.fa_std_softmax.restype = c_int
     lib.fa_bwd_workspace_size.argtypes = [c_int] * 5
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_validate_cu_seqlens.argtypes = [vp, c_int, c_int, c_int, vp]
+    lib.fa_validate_cu_seqlens.restype = c_int
     lib.fa_device_error.argtypes = []
     lib.fa_device_error.restype = c_int
     lib.fa_clear_device_error.argtypes = []
@@ -102,36 +104,37 @@ def load(build_if_missing=True):
 
 # ------------------------------------------------------------ raw C entry points
 
-def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, total_tokens, stream):
-    return load().fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, int(causal), cu_seqlens,
+def fa_fwd(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, causal, cu_seqlens, total_tokens,
+           stream):
+    return load().fa_fwd(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, int(causal), cu_seqlens,
                          total_tokens, stream)
 
 
-def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+def fa_bwd(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
            scale, causal, cu_seqlens, total_tokens, stream):
-    return load().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq,
+    return load().fa_bwd(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq,
                          Hkv, N, d, scale, int(causal), cu_seqlens, total_tokens, stream)
 
 
-def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal, cu_seqlens,
-                   total_tokens, stream):
+def fa_bwd_noalloc(q, k, v, o, lse, o_lo, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale, causal,
+                   cu_seqlens, total_tokens, stream):
     """Backward through the library's fixed scratch array (no allocation by
     the library or by this binding); see include/fa.h for its limits."""
-    return load().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
+    return load().fa_bwd_noalloc(q, k, v, o, lse, o_lo, dO, dq, dk, dv, B, Hq, Hkv, N, d, scale,
                                  int(causal), cu_seqlens, total_tokens, stream)
 
 
-def fa_fwd_blockmask(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, block_mask, mask_bs,
+def fa_fwd_blockmask(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, causal, block_mask, mask_bs,
                      mask_hs, stream):
-    return load().fa_fwd_blockmask(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, int(causal),
+    return load().fa_fwd_blockmask(q, k, v, o, lse, o_lo, B, Hq, Hkv, N, d, scale, int(causal),
                                    block_mask, mask_bs, mask_hs, stream)
 
 
-def fa_bwd_blockmask(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N,
-                     d, scale, causal, block_mask, mask_bs, mask_hs, stream):
-    return load().fa_bwd_blockmask(q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B,
-                                   Hq, Hkv, N, d, scale, int(causal), block_mask, mask_bs,
-                                   mask_hs, stream)
+def fa_bwd_blockmask(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace, workspace_bytes, B, Hq,
+                     Hkv, N, d, scale, causal, block_mask, mask_bs, mask_hs, stream):
+    return load().fa_bwd_blockmask(q, k, v, o, lse, o_lo, dO, dq, dk, dv, workspace,
+                                   workspace_bytes, B, Hq, Hkv, N, d, scale, int(causal),
+                                   block_mask, mask_bs, mask_hs, stream)
 
 
 def fa_decode(q, k_cache, v_cache, o, lse, cache_seqlens, B, Hq, Hkv, Lmax, d, scale, workspace,
@@ -152,6 +155,12 @@ def fa_std_softmax(s, p, lse, BH, N, scale, causal, stream):
 
 def fa_bwd_workspace_size(B, Hq, N, d, total_tokens):
     return load().fa_bwd_workspace_size(B, Hq, N, d, total_tokens)
+
+
+def fa_validate_cu_seqlens(cu_seqlens, B, N, total_tokens, stream):
+    """Enqueue the device-side check of a cu_seqlens array; its verdict is
+    read with fa_device_error() after a synchronise (see include/fa.h)."""
+    return load().fa_validate_cu_seqlens(cu_seqlens, B, N, total_tokens, stream)
 
 
 def fa_device_error():
@@ -216,8 +225,10 @@ def _check(t, name, dtype=torch.bfloat16):
 
 
 def attention_fwd(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen=None,
-                  out=None, lse=None):
-    """O, LSE = fa_fwd(q, k, v).  Dense [B, N, H, d] or varlen [total, H, d]."""
+                  out=None, lse=None, o_lo=None):
+    """O, LSE = fa_fwd(q, k, v).  Dense [B, N, H, d] or varlen [total, H, d].
+    o_lo: optional bf16 tensor shaped like q that receives O's rounding
+    residual (pass it to attention_bwd for an fp32-accurate D)."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, nm)
     B, Hq, Hkv, N, d, total = _shape(q, k, cu_seqlens, max_seqlen)
@@ -230,7 +241,11 @@ def attention_fwd(q, k, v, scale=None, causal=False, cu_seqlens=None, max_seqlen
                           dtype=torch.float32, device=q.device)
     if cu_seqlens is not None:
         _check(cu_seqlens, "cu_seqlens", torch.int32)
-    st = fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+    if o_lo is not None:
+        _check(o_lo, "o_lo")
+        if o_lo.shape != q.shape:
+            raise ValueError("o_lo must have q's shape")
+    st = fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(o_lo), B, Hq, Hkv, N, d,
                 float(scale), causal, _ptr(cu_seqlens), total, _stream())
     if st != FA_OK:
         raise FAError("fa_fwd", st)
@@ -245,10 +260,13 @@ def workspace_for(q, k, cu_seqlens=None, max_seqlen=None):
 
 
 def attention_bwd(q, k, v, out, lse, dout, scale=None, causal=False, cu_seqlens=None,
-                  max_seqlen=None, workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV = fa_bwd(...), recomputing P from the forward's LSE."""
+                  max_seqlen=None, workspace=None, dq=None, dk=None, dv=None, o_lo=None):
+    """dQ, dK, dV = fa_bwd(...), recomputing P from the forward's LSE.
+    o_lo: the forward's rounding residual of O, if it was written."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, nm)
+    if o_lo is not None:
+        _check(o_lo, "o_lo")
     _check(lse, "lse", torch.float32)
     B, Hq, Hkv, N, d, total = _shape(q, k, cu_seqlens, max_seqlen)
     if scale is None:
@@ -259,30 +277,31 @@ def attention_bwd(q, k, v, out, lse, dout, scale=None, causal=False, cu_seqlens=
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
-                _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, N, d, float(scale),
-                causal, _ptr(cu_seqlens), total, _stream())
+    st = fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(o_lo), _ptr(dout), _ptr(dq),
+                _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, N, d,
+                float(scale), causal, _ptr(cu_seqlens), total, _stream())
     if st != FA_OK:
         raise FAError("fa_bwd", st)
     return dq, dk, dv
 
 
 class Attention(torch.autograd.Function):
-    """Autograd wrapper: forward saves Q, K, V, O and LSE (O(N) memory) and
-    the backward recomputes P in fa_bwd."""
+    """Autograd wrapper: forward saves Q, K, V, O, O's rounding residual and
+    LSE (O(N) memory) and the backward recomputes P in fa_bwd."""
 
     @staticmethod
     def forward(ctx, q, k, v, scale, causal, cu_seqlens, max_seqlen):
-        o, lse = attention_fwd(q, k, v, scale, causal, cu_seqlens, max_seqlen)
-        ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
+        o_lo = torch.empty_like(q)
+        o, lse = attention_fwd(q, k, v, scale, causal, cu_seqlens, max_seqlen, o_lo=o_lo)
+        ctx.save_for_backward(q, k, v, o, lse, o_lo, cu_seqlens)
         ctx.scale, ctx.causal, ctx.max_seqlen = scale, causal, max_seqlen
         return o
 
     @staticmethod
     def backward(ctx, do):
-        q, k, v, o, lse, cu = ctx.saved_tensors
+        q, k, v, o, lse, o_lo, cu = ctx.saved_tensors
         dq, dk, dv = attention_bwd(q, k, v, o, lse, do.contiguous(), ctx.scale, ctx.causal,
-                                   cu, ctx.max_seqlen)
+                                   cu, ctx.max_seqlen, o_lo=o_lo)
         return dq, dk, dv, None, None, None, None
 
 
@@ -304,7 +323,8 @@ def _mask_strides(block_mask, B, Hkv, N):
     return sb, sh
 
 
-def attention_fwd_blockmask(q, k, v, block_mask, scale=None, causal=False, out=None, lse=None):
+def attention_fwd_blockmask(q, k, v, block_mask, scale=None, causal=False, out=None, lse=None,
+                            o_lo=None):
     """O, LSE of block-sparse attention (fa_fwd_blockmask): dense [B, N, H, d]
     inputs; block_mask [1 or B, 1 or Hkv, nt, nt] uint8 on the device,
     nt = ceil(N / 128), nonzero = the 128 x 128 tile is computed."""
@@ -317,15 +337,17 @@ def attention_fwd_blockmask(q, k, v, block_mask, scale=None, causal=False, out=N
         scale = d ** -0.5
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    st = fa_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
-                          float(scale), causal, _ptr(block_mask), sb, sh, _stream())
+    if o_lo is not None:
+        _check(o_lo, "o_lo")
+    st = fa_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(o_lo), B, Hq, Hkv,
+                          N, d, float(scale), causal, _ptr(block_mask), sb, sh, _stream())
     if st != FA_OK:
         raise FAError("fa_fwd_blockmask", st)
     return out, lse
 
 
 def attention_bwd_blockmask(q, k, v, out, lse, dout, block_mask, scale=None, causal=False,
-                            workspace=None):
+                            workspace=None, o_lo=None):
     """dQ, dK, dV of block-sparse attention (fa_bwd_blockmask)."""
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, nm)
@@ -339,9 +361,12 @@ def attention_bwd_blockmask(q, k, v, out, lse, dout, block_mask, scale=None, cau
         workspace = torch.empty(fa_bwd_workspace_size(B, Hq, N, d, B * N), dtype=torch.uint8,
                                 device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    st = fa_bwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
-                          _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, Hq, Hkv, N,
-                          d, float(scale), causal, _ptr(block_mask), sb, sh, _stream())
+    if o_lo is not None:
+        _check(o_lo, "o_lo")
+    st = fa_bwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(o_lo), _ptr(dout),
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B,
+                          Hq, Hkv, N, d, float(scale), causal, _ptr(block_mask), sb, sh,
+                          _stream())
     if st != FA_OK:
         raise FAError("fa_bwd_blockmask", st)
     return dq, dk, dv

@@ -20,6 +20,9 @@
  *                  (d contiguous; rows of one token are Hq*d or Hkv*d apart)
  *   lse          : fp32, dense [B][Hq][N] or varlen [Hq][total]; natural
  *                  log in the scaled-logit domain
+ *   o_lo         : optional bf16 in q's layout (NULL: none): the forward's
+ *                  second output, O - bf16(O) rounded to bf16, which the
+ *                  backward adds to o when it forms D = rowsum(dO o O)
  *   B            : batch size; with cu_seqlens, the number of sequences
  *   Hq, Hkv      : query / key-value heads; Hq % Hkv == 0.  Query head h
  *                  reads key/value head h / (Hq / Hkv) (grouped-query
@@ -32,7 +35,12 @@
  *   causal       : nonzero -> key j is masked for query i when j > i
  *                  (positions counted from the start of each sequence)
  *   cu_seqlens   : NULL for dense inputs, else device int32[B+1] prefix sums
- *                  of the sequence lengths (padding-free batches)
+ *                  of the sequence lengths (padding-free batches).  The
+ *                  kernels clamp every range they read from it to
+ *                  [0, total_tokens], so a corrupt array (not starting at 0,
+ *                  decreasing, past total_tokens, a length above N) gives
+ *                  undefined results but no access outside the caller's
+ *                  buffers; fa_validate_cu_seqlens() reports such an array
  *   total_tokens : with cu_seqlens, cu_seqlens[B] (the caller's allocation
  *                  size); ignored for dense inputs
  *   stream       : CUDA stream the kernels are enqueued on
@@ -45,8 +53,9 @@
  * holds until exit, whose device address is cached per device and whose
  * contents persist from call to call (overlapping fa_bwd_noalloc calls race
  * on it).  Host-side state is limited to settings (wait limit, profiling
- * events), cached driver entry points and that per-device address.  All pointers are
- * device pointers on one device and must be 16-byte aligned.  The kernels
+ * events), cached driver entry points and that per-device address.  All
+ * pointers are device pointers on one device and must be 16-byte aligned
+ * (a NULL optional pointer included).  The kernels
  * run on the device that owns q: if it is not the calling thread's current
  * device, the call makes it current (this also gives a thread that has not
  * used CUDA before a context).  A host pointer for q is FA_ERR_INVALID_ARG.
@@ -78,12 +87,18 @@ typedef enum {
 /*
  * Forward: O = softmax(scale Q K^T + mask) V and LSE.
  * Outputs o (bf16, q's layout) and lse (fp32, layout above) are fully
- * written for every valid token row; nothing else is touched.
+ * written for every valid token row; nothing else is touched.  When o_lo is
+ * not NULL it receives, for the same rows, the rounding residual of o (the
+ * fp32 result minus its bf16 rounding, itself rounded to bf16); o + o_lo
+ * then carries about 16 significant bits of O.  Pass it on to fa_bwd: its
+ * D = rowsum(dO o O) is otherwise formed from bf16 O, whose rounding error
+ * reaches dK through the term -scale P_ij D_i Q_i (large for query rows of
+ * large norm).  o_lo must not alias o.
  * Cites: "注意力机制基础" 2.1 (definition), "FlashAttention优化" 3.1 (tiling),
  * 3.2.1 (online softmax statistics m and l), paper review 方法 items 1-2
  * (tiles stay on chip, output rescale by exp(m_old - m_new)).
  */
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* o_lo,
                  int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                  const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
@@ -97,7 +112,8 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens);
 /*
  * Backward by recomputation (paper review, 方法 item 3): P is rebuilt from
  * Q, K and the forward's LSE; no S or P was stored.  Inputs q, k, v, o, lse,
- * dO as produced for / by fa_fwd with the same sizes; outputs dq (q's
+ * o_lo (optional, NULL if the forward did not write it), dO as produced
+ * for / by fa_fwd with the same sizes; outputs dq (q's
  * layout), dk and dv (k's layout; summed over the query heads of each
  * group).  `workspace` is caller-owned device memory of at least
  * fa_bwd_workspace_size() bytes, 256-byte aligned; its contents on entry do
@@ -105,9 +121,10 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens);
  * may differ between runs; dK and dV are deterministic.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                 const void* dO, void* dq, void* dk, void* dv, void* workspace,
-                 size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, float scale,
-                 int causal, const int* cu_seqlens, int total_tokens, cudaStream_t stream);
+                 const void* o_lo, const void* dO, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d,
+                 float scale, int causal, const int* cu_seqlens, int total_tokens,
+                 cudaStream_t stream);
 
 /*
  * Block-sparse attention: the same forward and backward with every (query,
@@ -129,14 +146,14 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * workspace size (fa_bwd_workspace_size with total_tokens = B * N).
  */
 fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o, float* lse,
-                           int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-                           const unsigned char* block_mask, long mask_batch_stride,
+                           void* o_lo, int B, int Hq, int Hkv, int N, int d, float scale,
+                           int causal, const unsigned char* block_mask, long mask_batch_stride,
                            long mask_head_stride, cudaStream_t stream);
 
 fa_status fa_bwd_blockmask(const void* q, const void* k, const void* v, const void* o,
-                           const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                           void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
-                           int N, int d, float scale, int causal,
+                           const float* lse, const void* o_lo, const void* dO, void* dq,
+                           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                           int Hq, int Hkv, int N, int d, float scale, int causal,
                            const unsigned char* block_mask, long mask_batch_stride,
                            long mask_head_stride, cudaStream_t stream);
 
@@ -171,8 +188,8 @@ fa_status fa_bwd_blockmask(const void* q, const void* k, const void* v, const vo
  *    them) race on the array and give wrong results: serialise them.
  */
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
-                         const float* lse, const void* dO, void* dq, void* dk, void* dv, int B,
-                         int Hq, int Hkv, int N, int d, float scale, int causal,
+                         const float* lse, const void* o_lo, const void* dO, void* dq, void* dk,
+                         void* dv, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                          const int* cu_seqlens, int total_tokens, cudaStream_t stream);
 
 /*
@@ -230,8 +247,25 @@ fa_status fa_std_softmax(const void* s, void* p, float* lse, int BH, int N, floa
                          int causal, cudaStream_t stream);
 
 /*
+ * Checks a cu_seqlens array on the device (one small kernel on `stream`,
+ * reading cu_seqlens[0..B] only): cu[0] == 0, cu non-decreasing, every
+ * length cu[b+1] - cu[b] at most N, and cu[B] <= total_tokens.  The first
+ * failing rule (in that order) is recorded in the device error word as
+ * 0x501, 0x502, 0x503 or 0x504, read by fa_device_error() after the caller
+ * synchronises; nothing is recorded for a valid array.  The check is
+ * optional: with the environment variable FA_DEBUG_VALIDATE set, every
+ * varlen fa_fwd / fa_bwd call runs it first on its own stream.  No
+ * counterpart on the pages; padding-free batches are the paper review's
+ * "消除 padding".  Returns FA_ERR_INVALID_ARG for a NULL or misaligned
+ * pointer or negative sizes, FA_ERR_CUDA if the launch fails.
+ */
+fa_status fa_validate_cu_seqlens(const int* cu_seqlens, int B, int N, int total_tokens,
+                                 cudaStream_t stream);
+
+/*
  * Device-side error word shared by all kernels of the library: 0 when no
- * wait has timed out since the last fa_clear_device_error().  Reads device
+ * wait has timed out (and no validation failed) since the last
+ * fa_clear_device_error().  Reads device
  * memory synchronously on the current device; call after synchronising.
  * Returns -1 if the read itself fails.
  */

@@ -8,7 +8,9 @@ The arithmetic lives in ``attention_oracle.c`` (plain fp64 C, OpenMP over
 independent problems); this module only marshals numpy arrays into it.  See
 that file's header for the definitions it follows and for which page passage
 each one cites.  ``brute.py`` is a second, fully independent pure-Python
-implementation for tiny shapes.
+implementation for tiny shapes.  ``columns.py`` holds the key-column sampler
+(dK, dV of selected key rows at sizes where the full backward is too slow),
+written with fp64 torch matrix products on the CPU.
 """
 import ctypes
 import os
@@ -16,6 +18,7 @@ import os
 import numpy as np
 
 from . import build as _build
+from .columns import attention_cols  # noqa: F401  (key-column sampler, torch fp64)
 
 _lib = None
 

@@ -14,11 +14,13 @@ from exact_io_aware_67_b200 import ops
 TOL_MAX = 2e-2
 TOL_MEAN = 2e-3
 TOL_LSE = 1e-3
-# dK of workloads with one query row scaled by 8: D = rowsum(dO o O) is formed
-# from the bf16-rounded O, and its rounding error reaches dK_j through the
-# term -scale P_ij D_i Q_i, where the scaled row Q_i is 8x larger than the
-# rest.  Measured worst case 6.2e-2 at N=1024, d=128; bound stated here.
-TOL_DK_X8 = 1e-1
+
+# Entries held to more than TOL_MAX, one record per assert_close call that had
+# any: (name, count, smallest |ref| among them, largest allowance).  Only an
+# entry whose oracle value is itself farther than TOL_MAX from every bf16
+# number (|ref| >= 8) is held to TOL_MAX plus that distance; the count is
+# printed and kept here so that the tests report it.
+LOOSENED = []
 
 
 def f64(t):
@@ -42,20 +44,25 @@ def max_seqlen(inp):
 
 
 def gpu_fwd(inp, dev=None):
-    dev = dev or to_dev(inp)
+    """O, LSE through fa_fwd; O's rounding residual goes to dev["o_lo"]
+    (the backward reads it from there, as a training step would)."""
+    dev = dev if dev is not None else to_dev(inp)
     w = inp.workload
+    dev["o_lo"] = torch.empty_like(dev["q"])
     o, lse = ops.attention_fwd(dev["q"], dev["k"], dev["v"], w.scale, w.causal, dev["cu"],
-                               max_seqlen(inp) if dev["cu"] is not None else None)
+                               max_seqlen(inp) if dev["cu"] is not None else None,
+                               o_lo=dev["o_lo"])
     torch.cuda.synchronize()
     return o, lse
 
 
 def gpu_bwd(inp, o, lse, dev=None):
-    dev = dev or to_dev(inp)
+    dev = dev if dev is not None else to_dev(inp)
     w = inp.workload
     dq, dk, dv = ops.attention_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["dout"], w.scale,
                                    w.causal, dev["cu"],
-                                   max_seqlen(inp) if dev["cu"] is not None else None)
+                                   max_seqlen(inp) if dev["cu"] is not None else None,
+                                   o_lo=dev.get("o_lo"))
     torch.cuda.synchronize()
     return dq, dk, dv
 
@@ -88,9 +95,13 @@ def rounding_distance(ref):
 
 
 def assert_close(name, got, ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN, bf16_out=True):
-    """Elementwise |got - ref| <= tol_max (+ the oracle value's own distance
-    to the nearest bf16 number when the output is stored in bf16: no bf16
-    output can be closer than that), and mean |got - ref| <= tol_mean."""
+    """Elementwise |got - ref| <= tol_max and mean |got - ref| <= tol_mean.
+
+    For a bf16 output, an entry whose oracle value lies farther than tol_max
+    from the nearest bf16 number (|ref| >= 8 at tol_max = 2e-2) cannot meet
+    tol_max in any bf16 result; such an entry alone is held to tol_max plus
+    that distance, and how many there were is printed and recorded in
+    LOOSENED.  Every other entry is held to tol_max."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
@@ -98,16 +109,26 @@ def assert_close(name, got, ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN, bf16_out=Tr
     mx, mn = errors(got, ref)
     if got.size == 0:
         return mx, mn
-    bound = tol_max + (rounding_distance(ref) if bf16_out else 0.0)
-    if np.any(np.abs(got - ref) > bound):
-        err = np.abs(got - ref)
-        w = np.unravel_index(np.argmax(err), err.shape)
+    err = np.abs(got - ref)
+    bound = np.full(ref.shape, tol_max)
+    if bf16_out:
+        floor = rounding_distance(ref)
+        loose = floor > tol_max
+        if np.any(loose):
+            bound = np.where(loose, tol_max + floor, tol_max)
+            rec = (name, int(loose.sum()), float(np.abs(ref[loose]).min()),
+                   float(bound[loose].max()))
+            LOOSENED.append(rec)
+            print("%s: %d entries with |ref| >= %.3g held to %.1e + their bf16 rounding "
+                  "distance (largest bound %.3e)" % rec)
+    if np.any(err > bound):
+        w = np.unravel_index(np.argmax(err - bound), err.shape)
         bad = err > bound
         raise AssertionError(
-            "%s max-abs error %.3e > %.1e (+rounding distance) (mean %.3e) at %s: got %.5f "
+            "%s error %.3e over its bound %.3e at %s (max-abs %.3e, mean %.3e): got %.5f "
             "ref %.5f; max|ref| %.3f; bf16 floor %.3e; entries over the bound: %d of %d, their "
-            "min |ref| %.3f" % (name, mx, tol_max, mn, w, got[w], ref[w], np.abs(ref).max(),
-                                bf16_floor(ref), int(bad.sum()), err.size,
+            "min |ref| %.3f" % (name, err[w], bound[w], w, mx, mn, got[w], ref[w],
+                                np.abs(ref).max(), bf16_floor(ref), int(bad.sum()), err.size,
                                 float(np.abs(ref[bad]).min())))
     if tol_mean is not None:
         assert mn <= tol_mean, "%s mean-abs error %.3e > %.1e" % (name, mn, tol_mean)

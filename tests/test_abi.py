@@ -39,18 +39,20 @@ def test_status_strings(lib):
 
 def _fwd(**kw):
     a = dict(q=ctypes.c_void_p(4096), k=ctypes.c_void_p(4096), v=ctypes.c_void_p(4096),
-             o=ctypes.c_void_p(4096), lse=ctypes.c_void_p(4096), B=1, Hq=2, Hkv=1, N=128, d=64,
-             scale=0.125, causal=0, cu_seqlens=None, total_tokens=0, stream=None)
+             o=ctypes.c_void_p(4096), lse=ctypes.c_void_p(4096), o_lo=None, B=1, Hq=2, Hkv=1,
+             N=128, d=64, scale=0.125, causal=0, cu_seqlens=None, total_tokens=0, stream=None)
     a.update(kw)
-    return ops.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["N"],
-                      a["d"], a["scale"], a["causal"], a["cu_seqlens"], a["total_tokens"],
-                      a["stream"])
+    return ops.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["o_lo"], a["B"], a["Hq"],
+                      a["Hkv"], a["N"], a["d"], a["scale"], a["causal"], a["cu_seqlens"],
+                      a["total_tokens"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(d=96), 2), (dict(d=256), 2), (dict(Hq=3, Hkv=2), 1), (dict(Hkv=0), 1),
     (dict(N=0), 1), (dict(B=-1), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1),
     (dict(q=None), 1), (dict(o=ctypes.c_void_p(4100)), 1),
+    (dict(o_lo=ctypes.c_void_p(4100)), 1),                        # misaligned residual
+    (dict(o_lo=ctypes.c_void_p(4096)), 1),                        # residual aliasing o
     (dict(cu_seqlens=ctypes.c_void_p(4096), total_tokens=-1), 1),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, expect):
@@ -68,7 +70,7 @@ def test_bwd_workspace_checks(lib):
     assert need >= 512 * 4 * 128 * 4 + 512 * 4 * 4
     assert ops.fa_bwd_workspace_size(1, 1, 1, 96, 1) == 0
     p = ctypes.c_void_p(4096)
-    args = [p] * 9
+    args = [p] * 5 + [None] + [p] * 4     # no residual of O
     st = ops.fa_bwd(*args, ctypes.c_void_p(4096), 1024, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
                     None)
     assert st == 3
@@ -77,6 +79,10 @@ def test_bwd_workspace_checks(lib):
     st = ops.fa_bwd(*args, ctypes.c_void_p(4096 + 16), need, 2, 4, 4, 256, 128, 0.1, 1, None, 0,
                     None)
     assert st == 3   # workspace must be 256-byte aligned
+    # a misaligned optional residual is rejected before the workspace check
+    st = ops.fa_bwd(*([p] * 5), ctypes.c_void_p(4104), *([p] * 4), ctypes.c_void_p(4096), need,
+                    2, 4, 4, 256, 128, 0.1, 1, None, 0, None)
+    assert st == 1
 
 
 def test_build_command_targets_sm100a():
@@ -123,7 +129,7 @@ def test_decode_rejects_bad_arguments(lib):
 def test_blockmask_rejects_bad_arguments(lib):
     p = ctypes.c_void_p(4096)
     m = ctypes.c_void_p(8192)
-    f = lambda **kw: ops.fa_fwd_blockmask(*([p] * 5), kw.get("B", 1), 2, 2, kw.get("N", 256),
+    f = lambda **kw: ops.fa_fwd_blockmask(*([p] * 5), None, kw.get("B", 1), 2, 2, kw.get("N", 256),
                                           kw.get("d", 64), 0.125, 0, kw.get("m", m),
                                           kw.get("sb", 0), kw.get("sh", 0), None)
     assert f(m=None) == 1
@@ -132,5 +138,6 @@ def test_blockmask_rejects_bad_arguments(lib):
     assert f(sb=-1) == 1
     assert f(B=0) == 0
     need = ops.fa_bwd_workspace_size(1, 2, 256, 64, 256)
-    g = ops.fa_bwd_blockmask(*([p] * 9), p, need, 1, 2, 2, 256, 64, 0.125, 1, None, 0, 0, None)
+    g = ops.fa_bwd_blockmask(*([p] * 5), None, *([p] * 4), p, need, 1, 2, 2, 256, 64, 0.125, 1,
+                             None, 0, 0, None)
     assert g == 1

@@ -27,9 +27,11 @@ def _run(inp, bm, causal):
     w = inp.workload
     dev = parity.to_dev(inp)
     bmd = torch.from_numpy(bm).cuda()
-    o, lse = ops.attention_fwd_blockmask(dev["q"], dev["k"], dev["v"], bmd, w.scale, causal)
+    o_lo = torch.empty_like(dev["q"])
+    o, lse = ops.attention_fwd_blockmask(dev["q"], dev["k"], dev["v"], bmd, w.scale, causal,
+                                         o_lo=o_lo)
     dq, dk, dv = ops.attention_bwd_blockmask(dev["q"], dev["k"], dev["v"], o, lse, dev["dout"],
-                                             bmd, w.scale, causal)
+                                             bmd, w.scale, causal, o_lo=o_lo)
     torch.cuda.synchronize()
     parity.no_device_error()
     return o, lse, dq, dk, dv

@@ -1,4 +1,5 @@
-"""The FMA-pipe exp2 used for part of the forward's exponentials (CPU).
+"""The FMA-pipe exp2 (packed pairs) used for part of the forward's
+exponentials (CPU).
 
 Simulates the kernel's fp32 operation sequence in numpy (clamp, rounding by
 the 1.5 * 2^23 constant, cubic in Horner form, exponent-field add) and checks
@@ -15,16 +16,24 @@ HDR = os.path.join(os.path.dirname(fit_exp2.__file__), "csrc", "sm100.cuh")
 
 
 def _coeffs_in_header():
+    """The cubic's coefficients as the packed kernel function states them
+    (each literal appears twice there, once per lane of the pair)."""
     txt = open(HDR).read()
-    body = txt[txt.index("float ex2_poly"):txt.index("__int_as_float(__float_as_int(p)")]
-    return [float(v.rstrip("f")) for v in re.findall(r"[0-9]\.[0-9]+e[-+][0-9]+f", body)]
+    body = txt[txt.index("float2 ex2_poly2"):txt.index("return make_float2(__int_as_float")]
+    vals = [float(v.rstrip("f")) for v in re.findall(r"[0-9]\.[0-9]+e[-+][0-9]+f", body)]
+    assert len(vals) == 8 and vals[0::2] == vals[1::2], vals
+    return vals[0::2]
 
 
 def _ex2_poly(x, c):
+    """The kernel's per-lane fp32 sequence: clamp, t = x + 1.5 2^23,
+    n = t - 1.5 2^23, f = fma(n, -1, x), cubic by three fmas, n added to the
+    exponent field."""
     f32 = np.float32
     x = np.maximum(x.astype(f32), f32(-125.0))
     t = (x + f32(12582912.0)).astype(f32)
-    f = (x - (t - f32(12582912.0)).astype(f32)).astype(f32)
+    n = (t - f32(12582912.0)).astype(f32)
+    f = (x.astype(np.float64) - n.astype(np.float64)).astype(f32)
     # fused multiply-adds, rounded once each (evaluate in fp64, round to fp32)
     p = (f.astype(np.float64) * c[3] + c[2]).astype(f32)
     p = (p.astype(np.float64) * f + c[1]).astype(f32)

@@ -2,12 +2,18 @@
 configuration the benchmark times (dense layout, default wait limit).
 
 The oracle cannot afford every element at these sizes, so each workload is
-checked three ways:
+checked four ways:
   * whole key/value groups (all their query heads) element by element where
-    the fp64 oracle finishes in seconds (N = 4096);
+    the fp64 oracle finishes in seconds or tens of seconds (N = 4096, and
+    heads 0 and 15 at N = 16384);
   * sampled query rows on every head -- O, LSE and dQ of a row depend only
     on that row, so the oracle computes them one by one (O(N d) per row);
     the rows scaled by 8 are always in the sample;
+  * sampled key rows on every key/value head -- dK and dV of a key row
+    depend on every query row's LSE and D, so the oracle's column sampler
+    computes those row statistics by the definition and then the sampled
+    columns; the sample always holds the first and last key rows, keys in
+    the diagonal tile of each x8 query row and the keys that row weighs most;
   * gradient invariants on every head: sum_j dK_j = 0 (each row of dS sums
     to 0) and sum_j dV_j = sum over the group of sum_i dO_i (each row of P
     sums to 1), up to the bf16 rounding of the outputs.
@@ -47,9 +53,12 @@ def _group_reference(inp, b, hk):
     heads = list(range(hk * g, (hk + 1) * g))
     k, v = _head(inp.k, b, hk), _head(inp.v, b, hk)
 
+    # one head per pool thread; a lone head gets all the oracle's threads
+    nth = 1 if len(heads) > 1 else 0
+
     def one(h):
         return oracle.attention_bwd(_head(inp.q, b, h), k, v, _head(inp.dout, b, h), w.scale,
-                                    w.causal, nthreads=1)
+                                    w.causal, nthreads=nth)
 
     with cf.ThreadPoolExecutor(len(heads)) as ex:
         res = list(ex.map(one, heads))
@@ -96,6 +105,58 @@ def _check_rows(inp, outs, nrows, seed=0):
                                     ref["dq"])
 
 
+def _key_sample(inp, b, hk, nrand, rng):
+    """Key rows of (sequence b, kv head hk) to check: first and last rows,
+    tile edges, seeded random rows, and for each x8 query row i of the group
+    the keys of its diagonal tile up to i plus the keys it weighs most (the
+    largest q_i . k_j over j <= i), where its dS is largest."""
+    w = inp.workload
+    N = w.N
+    keys = {0, 1, 127, 128, N // 2, N - 1}
+    keys |= set(int(x) for x in rng.integers(0, N, nrand))
+    if inp.x8_rows is not None:
+        g = w.Hq // w.Hkv
+        kf = inp.k[b, :, hk].float()
+        for h in range(hk * g, (hk + 1) * g):
+            i = int(inp.x8_rows[b, h])
+            t0 = 128 * (i // 128)
+            keys |= {t0, i, (t0 + i) // 2}
+            lim = i + 1 if w.causal else N
+            logit = kf[:lim] @ inp.q[b, i, h].float()
+            keys |= set(int(x) for x in torch.topk(logit, min(3, lim)).indices)
+    return sorted(keys)
+
+
+def _check_cols(inp, outs, nrand, seed=0):
+    """dK and dV of sampled key rows on every kv head against the oracle's
+    column sampler (summed over each group's query heads)."""
+    o, lse, dq, dk, dv = outs
+    w = inp.workload
+    rng = np.random.default_rng(seed)
+    g = w.Hq // w.Hkv
+    for b in range(w.B):
+        for hk in range(w.Hkv):
+            keys = _key_sample(inp, b, hk, nrand, rng)
+            heads = slice(hk * g, (hk + 1) * g)
+            f = lambda t, hs: t[b:b + 1, :, hs].float().numpy().astype(np.float64)
+            cols = np.array([[0, 0, j] for j in keys])
+            ref = oracle.attention_cols(f(inp.q, heads), f(inp.k, slice(hk, hk + 1)),
+                                        f(inp.v, slice(hk, hk + 1)), f(inp.dout, heads), cols,
+                                        w.scale, w.causal)
+            parity.assert_close("dK cols b%d kv%d" % (b, hk), parity.f64(dk[b, keys, hk]),
+                                ref["dk"])
+            parity.assert_close("dV cols b%d kv%d" % (b, hk), parity.f64(dv[b, keys, hk]),
+                                ref["dv"])
+
+
+def _to_host(outs):
+    """Copy the GPU outputs to host memory and release the device copies."""
+    host = tuple(t.cpu() for t in outs)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return host
+
+
 def _check_invariants(inp, outs):
     o, lse, dq, dk, dv = outs
     w = inp.workload
@@ -127,17 +188,28 @@ def test_long_causal_n4096_x8row(d):
     inp = workloads.generate(workloads.WORKLOADS["long_causal_b1_h16_n4096_d%d_x8row" % d])
     outs = _run_gpu(inp)
     for hk in (0, 15):
-        _check_group(inp, outs, 0, hk, parity.TOL_DK_X8)
+        _check_group(inp, outs, 0, hk, parity.TOL_MAX)
     _check_rows(inp, outs, nrows=8)
     _check_invariants(inp, outs)
 
 
-@pytest.mark.parametrize("n", [16384, 65536])
 @pytest.mark.parametrize("d", [64, 128])
-def test_long_causal_x8row_sampled(n, d):
-    inp = workloads.generate(workloads.WORKLOADS["long_causal_b1_h16_n%d_d%d_x8row" % (n, d)])
+def test_long_causal_n16384_x8row(d):
+    inp = workloads.generate(workloads.WORKLOADS["long_causal_b1_h16_n16384_d%d_x8row" % d])
     outs = _run_gpu(inp)
-    _check_rows(inp, outs, nrows=6 if n == 16384 else 3)
     _check_invariants(inp, outs)
-    del outs
-    torch.cuda.empty_cache()
+    outs = _to_host(outs)
+    for hk in (0, 15):
+        _check_group(inp, outs, 0, hk, parity.TOL_MAX)
+    _check_rows(inp, outs, nrows=6)
+    _check_cols(inp, outs, nrand=8)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_long_causal_n65536_x8row(d):
+    inp = workloads.generate(workloads.WORKLOADS["long_causal_b1_h16_n65536_d%d_x8row" % d])
+    outs = _run_gpu(inp)
+    _check_invariants(inp, outs)
+    outs = _to_host(outs)
+    _check_rows(inp, outs, nrows=3)
+    _check_cols(inp, outs, nrand=6)

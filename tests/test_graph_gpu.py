@@ -28,9 +28,11 @@ def _inputs(varlen, seed):
 def _step(dev, inp, ws):
     w = inp.workload
     ms = parity.max_seqlen(inp) if dev["cu"] is not None else None
-    o, lse = ops.attention_fwd(dev["q"], dev["k"], dev["v"], w.scale, w.causal, dev["cu"], ms)
+    o_lo = torch.empty_like(dev["q"])
+    o, lse = ops.attention_fwd(dev["q"], dev["k"], dev["v"], w.scale, w.causal, dev["cu"], ms,
+                               o_lo=o_lo)
     dq, dk, dv = ops.attention_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["dout"], w.scale,
-                                   w.causal, dev["cu"], ms, workspace=ws)
+                                   w.causal, dev["cu"], ms, workspace=ws, o_lo=o_lo)
     return o, lse, dq, dk, dv
 
 

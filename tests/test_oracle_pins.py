@@ -245,6 +245,86 @@ def test_row_sample_matches_full():
         np.testing.assert_allclose(r["dq"][t], full["dq"][b, i, h], atol=1e-13)
 
 
+# ---------------------------------------------------------------- key-column sampler
+
+def _all_cols(B, Hkv, N):
+    return np.array([[b, h, j] for b in range(B) for h in range(Hkv) for j in range(N)])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,N,Hq,Hkv,d", [(2, 300, 4, 2, 16), (1, 517, 2, 1, 64),
+                                          (1, 700, 3, 3, 8)])
+def test_cols_match_full_backward(B, N, Hq, Hkv, d, causal):
+    """Every key row's dK, dV from the column sampler (torch fp64 products)
+    equals the C oracle's full backward; N spans several of its row blocks."""
+    rng = np.random.default_rng(B * N + d + causal)
+    q, k = rng.standard_normal((B, N, Hq, d)), rng.standard_normal((B, N, Hkv, d))
+    v, do = rng.standard_normal((B, N, Hkv, d)), rng.standard_normal((B, N, Hq, d))
+    full = oracle.attention_bwd(q, k, v, do, d ** -0.5, causal)
+    cols = _all_cols(B, Hkv, N)
+    got = oracle.attention_cols(q, k, v, do, cols, d ** -0.5, causal)
+    np.testing.assert_allclose(got["dk"], full["dk"][cols[:, 0], cols[:, 2], cols[:, 1]],
+                               rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["dv"], full["dv"][cols[:, 0], cols[:, 2], cols[:, 1]],
+                               rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_cols_varlen_match_full_backward(causal):
+    lengths = [5, 600, 1, 130]
+    Hq, Hkv, d = 4, 2, 8
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(cu[-1])
+    rng = np.random.default_rng(7 + causal)
+    q, k, v, do = (rng.standard_normal((T, H, d)) for H in (Hq, Hkv, Hkv, Hq))
+    full = oracle.attention_bwd(q, k, v, do, 0.3, causal, cu_seqlens=cu)
+    cols = np.array([[s, h, j] for s, L in enumerate(lengths) for h in range(Hkv)
+                     for j in range(L)])
+    got = oracle.attention_cols(q, k, v, do, cols, 0.3, causal, cu_seqlens=cu)
+    tok = cu[cols[:, 0]] + cols[:, 2]
+    np.testing.assert_allclose(got["dk"], full["dk"][tok, cols[:, 1]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["dv"], full["dv"][tok, cols[:, 1]], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_cols_match_brute_force(causal):
+    n, Hq, Hkv, d = 4, 2, 1, 3
+    rng = np.random.default_rng(31 + causal)
+    q, k = rng.standard_normal((1, n, Hq, d)), rng.standard_normal((1, n, Hkv, d))
+    v, do = rng.standard_normal((1, n, Hkv, d)), rng.standard_normal((1, n, Hq, d))
+    _, bdk, bdv = brute.backward(to_lists(q[0]), to_lists(k[0]), to_lists(v[0]),
+                                 to_lists(do[0]), 0.8, causal)
+    got = oracle.attention_cols(q, k, v, do, _all_cols(1, Hkv, n), 0.8, causal)
+    np.testing.assert_allclose(got["dk"], np.array(bdk)[:, 0], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(got["dv"], np.array(bdv)[:, 0], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_cols_finite_differences(causal):
+    """Central differences of L = sum(O o dO) (O from the C oracle's forward)
+    with respect to sampled K and V entries match the column sampler."""
+    N, Hq, Hkv, d = 11, 4, 2, 4
+    rng = np.random.default_rng(99 + causal)
+    q, k = rng.standard_normal((1, N, Hq, d)), rng.standard_normal((1, N, Hkv, d))
+    v, do = rng.standard_normal((1, N, Hkv, d)), rng.standard_normal((1, N, Hq, d))
+    scale = 0.5
+    cols = np.array([[0, 0, 0], [0, 1, 5], [0, 1, 10], [0, 0, 7]])
+    got = oracle.attention_cols(q, k, v, do, cols, scale, causal)
+    h = 1e-6
+    for t, (_, hk, j) in enumerate(cols):
+        for name, arr in (("dk", k), ("dv", v)):
+            for c in range(d):
+                a0 = arr[0, j, hk, c]
+                arr[0, j, hk, c] = a0 + h
+                lp = _loss(q, k, v, do, scale, causal)
+                arr[0, j, hk, c] = a0 - h
+                lm = _loss(q, k, v, do, scale, causal)
+                arr[0, j, hk, c] = a0
+                fd = (lp - lm) / (2 * h)
+                an = got[name][t, c]
+                assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, t, c, fd, an)
+
+
 # ---------------------------------------------------------------- library routine
 
 def _torch_reference(q, k, v, do, scale, causal):

@@ -26,7 +26,8 @@ def test_noalloc_rejects_problems_beyond_capacity():
     need = ops.fa_bwd_workspace_size(64, 64, 4096, 128, 64 * 4096)
     assert need > ops.FA_BWD_NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(4096)
-    st = ops.fa_bwd_noalloc(*([fake] * 9), 64, 64, 64, 4096, 128, 0.088, 1, None, 0, None)
+    st = ops.fa_bwd_noalloc(*([fake] * 5), None, *([fake] * 4), 64, 64, 64, 4096, 128, 0.088, 1,
+                            None, 0, None)
     assert st == 3   # FA_ERR_WORKSPACE
 
 
@@ -50,8 +51,8 @@ def test_noalloc_matches_workspace_entry_point_twice(varlen):
         dk = torch.full_like(dev["k"], float("nan"))
         dv = torch.full_like(dev["v"], float("nan"))
         st = ops.fa_bwd_noalloc(_p(dev["q"]), _p(dev["k"]), _p(dev["v"]), _p(o), _p(lse),
-                                _p(dev["dout"]), _p(dq), _p(dk), _p(dv), B, w.Hq, w.Hkv, N, w.d,
-                                w.scale, w.causal, _p(dev["cu"]), total, stream)
+                                _p(dev["o_lo"]), _p(dev["dout"]), _p(dq), _p(dk), _p(dv), B, w.Hq,
+                                w.Hkv, N, w.d, w.scale, w.causal, _p(dev["cu"]), total, stream)
         assert st == 0, ops.fa_status_string(st)
         torch.cuda.synchronize()
         parity.no_device_error()
