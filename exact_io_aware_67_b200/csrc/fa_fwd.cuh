@@ -76,11 +76,21 @@ static_assert(128 * (2 * FWD_REGS_SOFTMAX + FWD_REGS_CTRL) <= 65536 &&
               "register split");
 constexpr float RESCALE_LOG2 = 8.0f;
 // Pairs out of every 8 column pairs whose exp2 runs on the FMA pipe
-// (ex2_poly2, packed) instead of MUFU.
-#ifndef FA_EXP2_POLY_PAIRS
-#define FA_EXP2_POLY_PAIRS 0
-#endif
-constexpr int EXP2_POLY_PAIRS_OF_8 = FA_EXP2_POLY_PAIRS;
+// (ex2_poly2, packed) instead of MUFU.  Measured on B200 with the packed
+// loop (forward TFLOP/s for 0 / 1 / 2 / 3 pairs of 8):
+//   d = 64,  causal H=16 N=4096:   524 / 522 / 514 / 498
+//   d = 64,  causal H=16 N=16384:  740 / 720 / 697 / 667
+//   d = 128, GQA B=2 Hq=32 N=4096: 979 / 990 / 997 / 1001
+//   d = 128, causal H=16 N=65536 (power-capped; per 100 MHz of SM clock):
+//            69.9 / 72.6 / 72.4 / 71.3
+// At d = 64 the softmax's latency chain, not MUFU throughput, sets the pace
+// and the polynomial only lengthens it; at d = 128 the MUFU queue is shared
+// by both warpgroups between longer MMA phases and a quarter of the pairs on
+// the FMA pipe shortens it.
+template <int D>
+constexpr int exp2_poly_pairs_of_8() {
+  return D == 128 ? 2 : 0;
+}
 
 template <int D, bool CAUSAL, bool SPARSE = false>
 __global__ void __launch_bounds__(FWD_THREADS, 1)
@@ -465,7 +475,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
         tmem_wait_st();
       }
-      // p = 2^(x - m); EXP2_POLY_PAIRS_OF_8 pairs in every 8 use the FMA-pipe
+      // p = 2^(x - m); exp2_poly_pairs_of_8<D>() pairs in every 8 use the FMA-pipe
       // exp2, the rest MUFU.  P (bf16) goes to this row of the 128B-swizzled
       // K-major P tile: columns 0-63 and 64-127 are two 16 KB regions.
       uint8_t* prow = sP + (L::P_SMEM ? t * 32768 + (r >> 3) * 1024 + (r & 7) * 128 : 0);
@@ -481,7 +491,7 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
                                              __uint_as_float(s[32 * cc + 2 * i + 1])),
                                  c22, nm2);
           float2 pp;
-          if ((i & 7) >= 8 - EXP2_POLY_PAIRS_OF_8)
+          if ((i & 7) >= 8 - exp2_poly_pairs_of_8<D>())
             pp = ex2_poly2(x);
           else
             pp = make_float2(ex2(x.x), ex2(x.y));

@@ -120,7 +120,7 @@ def assert_close(name, got, ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN, bf16_out=Tr
                    float(bound[loose].max()))
             LOOSENED.append(rec)
             print("%s: %d entries with |ref| >= %.3g held to %.1e + their bf16 rounding "
-                  "distance (largest bound %.3e)" % rec)
+                  "distance (largest bound %.3e)" % (rec[0], rec[1], rec[2], tol_max, rec[3]))
     if np.any(err > bound):
         w = np.unravel_index(np.argmax(err - bound), err.shape)
         bad = err > bound
