@@ -63,11 +63,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return f;
 }
 
-// Tensor map over a token-major bf16 tensor [batches][rows][heads][d]:
+// Tensor map over a token-major 16-bit tensor [batches][rows][heads][d]
+// (bf16 by default; the backward's fp16 operand copies use the same shape):
 // box = 64 d-elements (128 B, 128-byte swizzle) x 1 head x 128 rows.
 // Rows past `rows` read as zeros.
 bool encode_rows_map(CUtensorMap* m, const void* base, int d, int heads, long rows,
-                     int batches) {
+                     int batches,
+                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows,
@@ -77,7 +79,7 @@ bool encode_rows_map(CUtensorMap* m, const void* base, int d, int heads, long ro
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r =
-      enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+      enc(m, dtype, 4, const_cast<void*>(base), dims, strides, box,
           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -275,22 +277,17 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   st = check_mask(bm, cu_seqlens, N);
   if (st != FA_OK) return st;
   if (empty) return FA_OK;
-  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d, s.tokens(), s.varlen);
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, Hkv, N, d, s.tokens(), s.varlen);
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FA_ERR_WORKSPACE;
   st = bind_device_of(q);
   if (st != FA_OK) return st;
 
-  CUtensorMap mq, mk, mv, mdo;
-  if (!encode_rows_map(&mq, q, d, Hq, s.rows(), s.batches()) ||
-      !encode_rows_map(&mk, k, d, Hkv, s.rows(), s.batches()) ||
-      !encode_rows_map(&mv, v, d, Hkv, s.rows(), s.batches()) ||
-      !encode_rows_map(&mdo, dO, d, Hq, s.rows(), s.batches()))
-    return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
-
   fa::BwdParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.o_lo = static_cast<const __nv_bfloat16*>(o_lo);
   p.dout = static_cast<const __nv_bfloat16*>(dO);
@@ -313,6 +310,14 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
   p.bm_sh = bm.sh;
   p.bm_nt = (N + 127) / 128;
   fa::bwd_carve_workspace(p, workspace, s.tokens(), d);
+  // the main kernel's products read the fp16 copies the preprocess writes
+  CUtensorMap mq, mk, mv, mdo;
+  const CUtensorMapDataType f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  if (!encode_rows_map(&mq, p.q16, d, Hq, s.rows(), s.batches(), f16) ||
+      !encode_rows_map(&mk, p.k16, d, Hkv, s.rows(), s.batches(), f16) ||
+      !encode_rows_map(&mv, p.v16, d, Hkv, s.rows(), s.batches(), f16) ||
+      !encode_rows_map(&mdo, p.do16, d, Hq, s.rows(), s.batches(), f16))
+    return cuda_fail(cudaErrorInvalidValue, "tensor map encode");
   if (cu_seqlens != nullptr && debug_validate()) {
     const cudaError_t ev = launch_validate_cu(cu_seqlens, B, N, total_tokens, stream);
     if (ev != cudaSuccess) return cuda_fail(ev, "cu_seqlens validation launch");
@@ -346,9 +351,11 @@ fa_status fa_fwd_blockmask(const void* q, const void* k, const void* v, void* o,
 size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens) {
   if (B < 0 || Hq < 1 || N < 1 || (d != 64 && d != 128) || total_tokens < 0) return 0;
   // the size must serve a dense call (total_tokens = B * N) and a varlen
-  // call with the same numbers, so take the larger of the two layouts
-  const size_t a = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, false);
-  const size_t v = fa::bwd_workspace_bytes(B, Hq, N, d, (long)total_tokens, true);
+  // call with the same numbers, so take the larger of the two layouts; the
+  // key/value head count is not an argument, so the K and V copies are sized
+  // for Hkv = Hq, an upper bound for every grouping
+  const size_t a = fa::bwd_workspace_bytes(B, Hq, Hq, N, d, (long)total_tokens, false);
+  const size_t v = fa::bwd_workspace_bytes(B, Hq, Hq, N, d, (long)total_tokens, true);
   return a > v ? a : v;
 }
 
@@ -383,7 +390,7 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (st != FA_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
-  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d, s.tokens(), s.varlen);
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, Hkv, N, d, s.tokens(), s.varlen);
   if (need > (size_t)FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
   st = bind_device_of(q);
   if (st != FA_OK) return st;

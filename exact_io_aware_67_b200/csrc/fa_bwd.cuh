@@ -57,8 +57,22 @@
 
 namespace fa {
 
+// Power-of-two scales of the backward's fp16 operands and the factors that
+// undo them (written by bwd_pre_kernel, read by the main and dQ kernels).
+struct BwdScales {
+  float sq, sk, sv, sdo;   // Q, K, V, dO copies = fp16(x * s_x)
+  float sds;               // dS operand = fp16(dS * s_ds)
+  float c2p;               // scale * log2(e) / (s_q s_k): S of the fp16 product -> log2 units
+  float vdo_sds;           // s_ds / (s_v s_do): dP of the fp16 product -> s_ds units
+  float dv_mul;            // 1 / s_do
+  float dk_mul;            // scale / (s_ds s_q)
+  float dq_mul;            // scale / (s_ds s_k)
+};
+
 struct BwdParams {
   const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
   const __nv_bfloat16* o;
   const __nv_bfloat16* o_lo;   // optional bf16 rounding residual of O (nullptr: none)
   const __nv_bfloat16* dout;
@@ -68,6 +82,14 @@ struct BwdParams {
   __nv_bfloat16* dv;
   float* dpsum;      // D, same layout as lse
   float* dq_acc;     // fp32 dQ accumulator (layout above)
+  // fp16 copies of the product operands (token-major, like the originals)
+  __half* q16;
+  __half* k16;
+  __half* v16;
+  __half* do16;
+  float* absmax_part;   // [nabs][4]: per-block max |Q|, |K|, |V|, |dO|
+  int nabs;             // blocks of bwd_absmax_kernel
+  BwdScales* scales;
   long tile_slots;   // tile slots of the accumulator per head
   int order_chunk;   // (sequence, kv head) pairs per dispatch chunk (causal grid order)
   const int* cu_seqlens;
@@ -81,23 +103,62 @@ struct BwdParams {
   int bm_nt;
 };
 
-inline size_t bwd_dsum_bytes(int Hq, long tokens) {
-  return ((size_t)Hq * (size_t)tokens * 4 + 255) & ~(size_t)255;
-}
+constexpr int ABSMAX_MAX_BLOCKS = 2048;
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // number of 128-row tile slots of the dQ accumulator
 inline long bwd_tile_slots(int B, int N, long tokens, bool varlen) {
   return varlen ? (tokens + 127) / 128 + B : (long)B * ((N + 127) / 128);
 }
 
-inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d, long tokens, bool varlen) {
-  return bwd_dsum_bytes(Hq, tokens) + (size_t)bwd_tile_slots(B, N, tokens, varlen) * Hq * 128 * d * 4;
+// Workspace layout: D, the max-abs partials, the scale record, the fp16
+// copies of Q, K, V, dO, and the fp32 dQ accumulator, each 256-byte aligned.
+struct BwdWsLayout {
+  size_t dsum, part, scales, q16, k16, v16, do16, acc, total;
+};
+
+inline BwdWsLayout bwd_ws_layout(int B, int Hq, int Hkv, int N, int d, long tokens,
+                                 bool varlen) {
+  BwdWsLayout w{};
+  size_t off = 0;
+  w.dsum = off;
+  off += align256((size_t)Hq * (size_t)tokens * 4);
+  w.part = off;
+  off += align256((size_t)ABSMAX_MAX_BLOCKS * 4 * 4);
+  w.scales = off;
+  off += 256;
+  w.q16 = off;
+  off += align256((size_t)tokens * Hq * d * 2);
+  w.k16 = off;
+  off += align256((size_t)tokens * Hkv * d * 2);
+  w.v16 = off;
+  off += align256((size_t)tokens * Hkv * d * 2);
+  w.do16 = off;
+  off += align256((size_t)tokens * Hq * d * 2);
+  w.acc = off;
+  off += (size_t)bwd_tile_slots(B, N, tokens, varlen) * Hq * 128 * d * 4;
+  w.total = off;
+  return w;
 }
 
-inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int /*d*/) {
+inline size_t bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d, long tokens,
+                                  bool varlen) {
+  return bwd_ws_layout(B, Hq, Hkv, N, d, tokens, varlen).total;
+}
+
+inline void bwd_carve_workspace(BwdParams& p, void* ws, long tokens, int d) {
+  const BwdWsLayout w =
+      bwd_ws_layout(p.B, p.Hq, p.Hkv, p.N, d, tokens, p.cu_seqlens != nullptr);
   uint8_t* base = static_cast<uint8_t*>(ws);
-  p.dpsum = reinterpret_cast<float*>(base);
-  p.dq_acc = reinterpret_cast<float*>(base + bwd_dsum_bytes(p.Hq, tokens));
+  p.dpsum = reinterpret_cast<float*>(base + w.dsum);
+  p.absmax_part = reinterpret_cast<float*>(base + w.part);
+  p.scales = reinterpret_cast<BwdScales*>(base + w.scales);
+  p.q16 = reinterpret_cast<__half*>(base + w.q16);
+  p.k16 = reinterpret_cast<__half*>(base + w.k16);
+  p.v16 = reinterpret_cast<__half*>(base + w.v16);
+  p.do16 = reinterpret_cast<__half*>(base + w.do16);
+  p.dq_acc = reinterpret_cast<float*>(base + w.acc);
   p.tile_slots = bwd_tile_slots(p.B, p.N, tokens, p.cu_seqlens != nullptr);
 }
 
@@ -124,19 +185,140 @@ __device__ __forceinline__ long stat_index(const BwdParams& p, int b, int h, int
 }
 
 // ============================================================================
-// K2: D = rowsum(dO o O) and zeroing of the dQ accumulator
+// K1: per-block max |x| of Q, K, V and dO
 // ============================================================================
-// Grid-stride; 8 blocks of 256 threads fit on an SM at the 32 registers the
-// launch bound asks for, so the launch (8 blocks per SM) is a single wave.
+// The backward's five products run on fp16 operands: 11 significant bits for
+// P and dS instead of bf16's 8, which keeps dV and dK within 2e-2 of the
+// exact gradient where their magnitude reaches 4-8 (there bf16 output
+// rounding alone takes up to 1.6e-2 of that).  Each input gets an fp16 copy
+// scaled by a power of two that puts its largest magnitude just below 2^14,
+// so the copy is exact for every bf16 value in fp16's normal range and the
+// scales cancel exactly.  This kernel finds the largest magnitudes; the
+// preprocess combines the per-block partials.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_absmax_kernel(const BwdParams p, long tokens) {
+  __shared__ float red[8][4];
+  const long gtid = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  const long gstride = (long)gridDim.x * blockDim.x;
+  float mx[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const __nv_bfloat16* src = t == 0 ? p.q : t == 1 ? p.k : t == 2 ? p.v : p.dout;
+    const int heads = (t == 0 || t == 3) ? p.Hq : p.Hkv;
+    const long n8 = tokens * heads * (D / 8);
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    float m = 0.f;
+    for (long i = gtid; i < n8; i += gstride) {
+      const uint4 a = s4[i];
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = unpack_bf16(w[e]);
+        m = fmaxf(m, fmaxf(fabsf(x.x), fabsf(x.y)));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    mx[t] = m;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0)
+    for (int t = 0; t < 4; ++t) red[warp][t] = mx[t];
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    float m = 0.f;
+    for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w][threadIdx.x]);
+    p.absmax_part[blockIdx.x * 4 + threadIdx.x] = m;
+  }
+}
+
+// 2^(14 - e) for m < 2^e: the power of two that puts m just below 2^14
+// (1 for m = 0 or a non-finite m; the exponent is clamped to stay normal).
+__device__ __forceinline__ float fp16_pow2_scale(float m) {
+  if (!(m > 0.f) || !isfinite(m)) return 1.f;
+  int e;
+  frexpf(m, &e);
+  return ldexpf(1.f, max(-100, min(100, 14 - e)));
+}
+
+// The scales from the four maxima (every caller computes the same values).
+__device__ __forceinline__ BwdScales bwd_make_scales(const BwdParams& p, const float mx[4],
+                                                     int d) {
+  BwdScales sc;
+  sc.sq = fp16_pow2_scale(mx[0]);
+  sc.sk = fp16_pow2_scale(mx[1]);
+  sc.sv = fp16_pow2_scale(mx[2]);
+  sc.sdo = fp16_pow2_scale(mx[3]);
+  // |dS| <= P (|dP| + |D|) <= 2 d max|dO| max|V| (|O| <= max|V| row by row)
+  sc.sds = fp16_pow2_scale(2.f * (float)d * mx[3] * mx[2]);
+  sc.c2p = p.scale_log2 / (sc.sq * sc.sk);
+  sc.vdo_sds = sc.sds / (sc.sv * sc.sdo);
+  sc.dv_mul = 1.f / sc.sdo;
+  sc.dk_mul = p.scale / (sc.sds * sc.sq);
+  sc.dq_mul = p.scale / (sc.sds * sc.sk);
+  return sc;
+}
+
+// ============================================================================
+// K2: scales, fp16 operand copies, D = rowsum(dO o O), zeroed dQ accumulator
+// ============================================================================
+// Grid-stride; every block first combines the max-abs partials into the
+// scales (block 0 also stores them for the later kernels), then writes its
+// share of the four fp16 copies, D and the zeroed accumulator.
 template <int D>
 __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long tokens) {
+  __shared__ float red[8][4];
+  __shared__ BwdScales s_sc;
+  {
+    float mx[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = threadIdx.x; i < p.nabs; i += blockDim.x)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) mx[t] = fmaxf(mx[t], p.absmax_part[i * 4 + t]);
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        mx[t] = fmaxf(mx[t], __shfl_xor_sync(0xffffffffu, mx[t], off));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0)
+      for (int t = 0; t < 4; ++t) red[warp][t] = mx[t];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m[4];
+      for (int t = 0; t < 4; ++t) {
+        m[t] = 0.f;
+        for (int w = 0; w < 8; ++w) m[t] = fmaxf(m[t], red[w][t]);
+      }
+      s_sc = bwd_make_scales(p, m, D);
+      if (blockIdx.x == 0) *p.scales = s_sc;
+    }
+    __syncthreads();
+  }
+  const long gtid = blockIdx.x * (long)blockDim.x + threadIdx.x;
+  const long gstride = (long)gridDim.x * blockDim.x;
+  // the fp16 copies
+#pragma unroll 1
+  for (int t = 0; t < 4; ++t) {
+    const __nv_bfloat16* src = t == 0 ? p.q : t == 1 ? p.k : t == 2 ? p.v : p.dout;
+    __half* dst = t == 0 ? p.q16 : t == 1 ? p.k16 : t == 2 ? p.v16 : p.do16;
+    const float sx = t == 0 ? s_sc.sq : t == 1 ? s_sc.sk : t == 2 ? s_sc.sv : s_sc.sdo;
+    const int heads = (t == 0 || t == 3) ? p.Hq : p.Hkv;
+    const long n8 = tokens * heads * (D / 8);
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    for (long i = gtid; i < n8; i += gstride) {
+      const uint4 a = s4[i];
+      const float2 x0 = unpack_bf16(a.x), x1 = unpack_bf16(a.y);
+      const float2 x2 = unpack_bf16(a.z), x3 = unpack_bf16(a.w);
+      d4[i] = make_uint4(pack_f16(x0.x * sx, x0.y * sx), pack_f16(x1.x * sx, x1.y * sx),
+                         pack_f16(x2.x * sx, x2.y * sx), pack_f16(x3.x * sx, x3.y * sx));
+    }
+  }
   // zero the accumulator
   {
     float4* acc = reinterpret_cast<float4*>(p.dq_acc);
     const long n4 = p.tile_slots * p.Hq * 128 * (D / 4);
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4;
-         i += (long)gridDim.x * blockDim.x)
-      acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long i = gtid; i < n4; i += gstride) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // one group of D/8 lanes per (token, head) row; each lane reads 8 bf16
   constexpr int LPR = D / 8;            // lanes per row
@@ -145,8 +327,8 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
   const int sub = lane / LPR;
   const int li = lane % LPR;
   const long rows = tokens * p.Hq;
-  const long warp_global = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5;
-  const long nwarps = ((long)gridDim.x * blockDim.x) >> 5;
+  const long warp_global = gtid >> 5;
+  const long nwarps = gstride >> 5;
   for (long base = warp_global * RPW; base < rows; base += nwarps * RPW) {
     const long row = base + sub;
     float s = 0.f;
@@ -186,7 +368,7 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
 }
 
 // ============================================================================
-// K4: dQ = scale * accumulator -> bf16 [token][head][d]
+// K4: dQ = scale * accumulator / (s_ds s_k) -> bf16 [token][head][d]
 // ============================================================================
 // Persistent: a few blocks per SM stride over the (query tile, head,
 // sequence) items, item = (b * Hq + h) * nq + i; 256 threads turn one
@@ -202,6 +384,8 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long ite
   constexpr int LD = (D / 4) * RH / 256;       // float4 loads per thread and half
   __shared__ __align__(16) float tile[RH][D + 4];
   const int tid = threadIdx.x;
+  // the accumulator holds sum dS16 K16 = s_ds s_k sum dS K
+  const float mul = p.scales->dq_mul;
   for (long it = blockIdx.x; it < items; it += gridDim.x) {
     const int i = (int)(it % nq);
     const long bh = it / nq;
@@ -235,10 +419,10 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p, long ite
         const float4 y = *reinterpret_cast<const float4*>(&tile[rr][8 * ch + 4 - 4 * sw]);
         const float4 lo = sw ? y : x, hi = sw ? x : y;
         uint4 w;
-        w.x = pack_bf16(lo.x * p.scale, lo.y * p.scale);
-        w.y = pack_bf16(lo.z * p.scale, lo.w * p.scale);
-        w.z = pack_bf16(hi.x * p.scale, hi.y * p.scale);
-        w.w = pack_bf16(hi.z * p.scale, hi.w * p.scale);
+        w.x = pack_bf16(lo.x * mul, lo.y * mul);
+        w.y = pack_bf16(lo.z * mul, lo.w * mul);
+        w.z = pack_bf16(hi.x * mul, hi.y * mul);
+        w.w = pack_bf16(hi.z * mul, hi.w * mul);
         *reinterpret_cast<uint4*>(p.dq + ((tok0 + r0 + rr) * p.Hq + h) * D + 8 * ch) = w;
       }
       __syncthreads();
@@ -459,6 +643,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   if (warp == 12) {
     // ============================================================ producer
     const float kLog2e = 1.4426950408889634f;
+    const float sds = p.scales->sds;
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
 #pragma unroll
@@ -499,8 +684,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       do_issued = n + 1;
       // statistics of the 128 query rows, negated for the packed elementwise
-      // math: -LSE * log2(e) and -D; rows past the sequence end get -inf / 0
-      // so that their P and dS vanish.  The stage's previous readers are
+      // math: -LSE * log2(e) and -D * s_ds (dS goes to fp16 scaled by s_ds);
+      // rows past the sequence end get -inf / 0 so that their P and dS
+      // vanish.  The stage's previous readers are
       // done: they finished before dK of iteration n-2, which released
       // q_empty[s].
       float lv[4], dv[4];
@@ -517,7 +703,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const int r = lane + 32 * e;
         const bool valid = 128 * i + r < len;
         st[r] = valid ? -lv[e] * kLog2e : -INFINITY;
-        st[128 + r] = valid ? -dv[e] : 0.f;
+        st[128 + r] = valid ? -dv[e] * sds : 0.f;
       }
       mbar_arrive(st_full + s);
     }
@@ -532,9 +718,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   } else if (warp == 13) {
     // ============================================================ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_sq = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t id_kn = idesc_bf16_f32(128, D, false, true);      // dV, dK
-      constexpr uint32_t id_mn = idesc_bf16_f32(128, D, true, true);       // dQ
+      // every product takes both operands in fp16 (the scaled copies of Q, K,
+      // V, dO, and P and dS written as fp16 by the elementwise warps)
+      constexpr uint32_t id_sq = idesc_f16_f32(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t id_kn = idesc_f16_f32(128, D, false, true);      // dV, dK
+      constexpr uint32_t id_mn = idesc_f16_f32(128, D, true, true);       // dQ
       // descriptors built once; K-major views (LBO unused) and N/M-major
       // views (LBO = distance between 64-element blocks)
       const SDesc kK = sdesc_make(smem_u32(sK), 16, 1024);     // K, A of S^T
@@ -682,7 +870,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const uint32_t tDP = tmem + lane_off + L::T_DP + 64 * wg;
     const int kv_row = 128 * j + r;
     const bool kv_ok = kv_row < len;
-    const float c2 = p.scale_log2;
+    // S and dP of the fp16 products carry the operand scales: c2 maps S to
+    // log2 units, vdo_sds maps dP to the s_ds units of the stored -D s_ds
+    const float c2 = p.scales->c2p;
+    const float vdo_sds = p.scales->vdo_sds;
     // byte offset of this thread's row inside its 64-column dS region
     uint8_t* ds_row = sDS + wg * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
     bool ok = true;
@@ -730,8 +921,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(P[2 * c], P[2 * c + 1]);
-        tmem_st32(tS, pk);      // P^T (bf16) over the S columns just read
+        for (int c = 0; c < 32; ++c) pk[c] = pack_f16(P[2 * c], P[2 * c + 1]);
+        tmem_st32(tS, pk);      // P^T (fp16) over the S columns just read
         tmem_wait_st();
       }
       tc_fence_before();
@@ -748,15 +939,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_wait_ld32(dv);
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
-          // dS = P (dP - D) (the stats hold -D)
+          // dS s_ds = P (dP vdo_sds - D s_ds) (the stats hold -D s_ds)
           const float4 d4 = *reinterpret_cast<const float4*>(st + 128 + 64 * wg + 32 * hh + 4 * c4);
           const int c = 32 * hh + 4 * c4;
-          const float2 ds01 = make_float2(P[c] * (__uint_as_float(dv[4 * c4 + 0]) + d4.x),
-                                          P[c + 1] * (__uint_as_float(dv[4 * c4 + 1]) + d4.y));
-          const float2 ds23 = make_float2(P[c + 2] * (__uint_as_float(dv[4 * c4 + 2]) + d4.z),
-                                          P[c + 3] * (__uint_as_float(dv[4 * c4 + 3]) + d4.w));
-          dsp[16 * hh + 2 * c4] = pack_bf16(ds01.x, ds01.y);
-          dsp[16 * hh + 2 * c4 + 1] = pack_bf16(ds23.x, ds23.y);
+          const float2 ds01 = make_float2(
+              P[c] * fmaf(__uint_as_float(dv[4 * c4 + 0]), vdo_sds, d4.x),
+              P[c + 1] * fmaf(__uint_as_float(dv[4 * c4 + 1]), vdo_sds, d4.y));
+          const float2 ds23 = make_float2(
+              P[c + 2] * fmaf(__uint_as_float(dv[4 * c4 + 2]), vdo_sds, d4.z),
+              P[c + 3] * fmaf(__uint_as_float(dv[4 * c4 + 3]), vdo_sds, d4.w));
+          dsp[16 * hh + 2 * c4] = pack_f16(ds01.x, ds01.y);
+          dsp[16 * hh + 2 * c4 + 1] = pack_f16(ds23.x, ds23.y);
         }
       }
       // the previous dS tile must have been consumed by its dK and dQ products
@@ -779,7 +972,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (ok) {
       tc_fence_after();
       const uint32_t tcol = tmem + lane_off + (wg == 0 ? L::T_DV : L::T_DK);
-      const float mul = (wg == 0) ? 1.f : p.scale;
+      // undo the operand scales: dV carries s_do, dK carries s_ds s_q
+      const float mul = (wg == 0) ? p.scales->dv_mul : p.scales->dk_mul;
       __nv_bfloat16* dst = (wg == 0) ? p.dv : p.dk;
       const long t = (p.cu_seqlens != nullptr) ? (long)seq_start + kv_row : (long)b * p.N + kv_row;
       __nv_bfloat16* row_ptr = dst + (t * p.Hkv + hk) * (long)D;
@@ -820,7 +1014,17 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  bwd_pre_kernel<D><<<sms * 8, 256, 0, stream>>>(p, tokens);
+  // K1: max-abs partials (one per block), K2: scales, fp16 copies, D, zeroed
+  // accumulator
+  BwdParams pp = p;
+  pp.nabs = std::min(sms * 4, ABSMAX_MAX_BLOCKS);
+  bwd_absmax_kernel<D><<<pp.nabs, 256, 0, stream>>>(pp, tokens);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: absmax kernel launch\n");
+    return e;
+  }
+  bwd_pre_kernel<D><<<sms * 8, 256, 0, stream>>>(pp, tokens);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: pre kernel launch\n");
@@ -835,7 +1039,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
   // the step went from 910 to 951 TFLOP/s, mostly through a higher sustained
   // clock; at N=16384, d=64 (64 MiB, in L2 anyway) chunks of 5 were 3% slower
   // than one chunk.
-  BwdParams pc = p;
+  BwdParams pc = pp;
   {
     const long nkv = (p.N + 127) / 128;
     const long bh = (long)p.Hkv * p.B;
@@ -874,7 +1078,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     dq_blocks_cache.store(dq_blocks_per_sm, std::memory_order_relaxed);
   }
   const long g2 = std::min<long>(items, (long)sms * dq_blocks_per_sm);
-  bwd_dq_kernel<D><<<(unsigned)g2, 256, 0, stream>>>(p, items, nq);
+  bwd_dq_kernel<D><<<(unsigned)g2, 256, 0, stream>>>(pp, items, nq);
   return cudaGetLastError();
 }
 

@@ -30,10 +30,14 @@
 //    a thread owns one query row (TMEM lane), so row max and row sum are
 //    in-thread reductions.
 //  * Exponentials are exp2 with the scale folded in (x = s scale log2 e).
-//    The running max is only moved when the tile max exceeds it by more than
-//    RESCALE_LOG2 (factor 256); otherwise the stale max is kept for both O
-//    and l, which is exact because the final O / l uses the same reference.
-//    O in TMEM is then rescaled only for rows whose max moved.
+//    The running max moves whenever a tile's max exceeds it, so every P~ is
+//    at most 1 and the largest one of a row is exactly 1.  (Keeping a stale
+//    max until the tile max exceeds it by a factor 2^8, which saves O
+//    rescales, lets P~ reach 256; its bf16 rounding in P V then scales a
+//    row dominated by one key by up to 1 +- 2^-9 as a whole, which biases
+//    D = rowsum(dO o O) in the backward by about 2^-9 D and dK past the
+//    2e-2 bar on rows of large norm.)  O in TMEM is rescaled only for the
+//    rows whose max moved.
 //  * Causal attention skips every K/V tile above the diagonal; only the
 //    last tile of each Q tile is masked element-wise.  Variable-length
 //    batches mask key columns past the sequence end and never store rows
@@ -74,7 +78,9 @@ constexpr int FWD_REGS_CTRL = 72;       // warpgroup 2 after setmaxnreg.dec
 static_assert(128 * (2 * FWD_REGS_SOFTMAX + FWD_REGS_CTRL) <= 65536 &&
                   2 * (FWD_REGS_SOFTMAX - 168) * 128 == (168 - FWD_REGS_CTRL) * 128,
               "register split");
-constexpr float RESCALE_LOG2 = 8.0f;
+// How far (in log2 units) a tile's max must exceed the running max before
+// the max moves; see the header comment for why it is 0.
+constexpr float RESCALE_LOG2 = 0.0f;
 // Pairs out of every 8 column pairs whose exp2 runs on the FMA pipe
 // (ex2_poly2, packed) instead of MUFU.  Measured on B200 with the packed
 // loop (forward TFLOP/s for 0 / 1 / 2 / 3 pairs of 8):
@@ -457,20 +463,31 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       if (L::P_SMEM && j > 0) {
         // PV_t of the previous K/V tile must be done: it reads the P_t buffer
-        // and accumulates into O_t.  (With P in TMEM, S_t^j was issued after
-        // that PV, so s_full already implies it.)
+        // and accumulates into O_t, which the rescale below rewrites.  (With P
+        // in TMEM, S_t^j was issued after that PV, so s_full already implies
+        // it.)
         ok = __all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, wd, ERR_FWD_P_FREE));
         if (!ok) break;
         tc_fence_after();
       }
-      if (__any_sync(0xffffffffu, resc)) {
+      const bool rescaled = __any_sync(0xffffffffu, resc);
+      if (L::P_SMEM && rescaled) {
+        // d = 64: O_t *= alpha now, 32 columns at a time (the S registers are
+        // live; with P in shared memory the previous P V has already been
+        // waited for above)
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld32(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 v =
+                fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+            o[i] = __float_as_uint(v.x);
+            o[i + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(tO + 32 * c, o);
         }
         tmem_wait_st();
@@ -514,6 +531,27 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
         }
       }
       l += (la.x + la.y) + (lb.x + lb.y);
+      // d = 128: O_t *= alpha for the rows whose max moved (the warp does it
+      // if any of its rows did) after the exponentials, when the S registers
+      // are dead, so the whole row is loaded at once and scaled with packed
+      // multiplies; the P V product of this tile is released only afterwards.
+      if (!L::P_SMEM && rescaled) {
+        uint32_t o[D];
+        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + 32 * c, o + 32 * c);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_wait_ld32(o + 32 * c);
+#pragma unroll
+        for (int i = 0; i < D; i += 2) {
+          const float2 v =
+              fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+          o[i] = __float_as_uint(v.x);
+          o[i + 1] = __float_as_uint(v.y);
+        }
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_st32(tO + 32 * c, o + 32 * c);
+      }
       if constexpr (L::P_SMEM)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       else

@@ -104,8 +104,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * Bytes of device workspace fa_bwd needs: the fp32 row vector
- * D = rowsum(dO o O) and the fp32 dQ accumulator.  For dense inputs pass
- * total_tokens = B * N.  Returns 0 for invalid sizes.
+ * D = rowsum(dO o O), fp16 copies of Q, K, V and dO (the backward's products
+ * run on fp16 operands, see fa_bwd), a few KB of scale bookkeeping, and the
+ * fp32 dQ accumulator.  The K and V copies are sized for Hkv = Hq, so the
+ * figure holds for every grouping.  For dense inputs pass total_tokens =
+ * B * N.  Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens);
 
@@ -119,6 +122,16 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d, int total_tokens);
  * fa_bwd_workspace_size() bytes, 256-byte aligned; its contents on entry do
  * not matter.  dQ accumulates in fp32 by atomic addition, so its low bits
  * may differ between runs; dK and dV are deterministic.
+ * Precision: the five products of the backward take fp16 operands -- copies
+ * of Q, K, V and dO each scaled by a power of two that puts its largest
+ * magnitude just below 2^14 (exact for every bf16 value in fp16's normal
+ * range), and P and dS rounded to fp16 (dS with its own power-of-two scale
+ * from the bound |dS| <= 2 d max|dO| max|V|) -- with fp32 accumulation; the
+ * scales are undone exactly in the epilogues.  fp16's 11 significant bits
+ * keep dV and dK within 2e-2 of the exact gradient where bf16 operands (8
+ * bits) did not.  Four kernels run in order: a max-magnitude pass, the
+ * preprocess (copies, D, zeroed accumulator), the main kernel, the dQ
+ * conversion.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* o_lo, const void* dO, void* dq, void* dk, void* dv,

@@ -80,7 +80,7 @@ def test_o_residual_is_the_rounding_error_of_o():
     ref_o, _ = parity.oracle_fwd(inp)
     e_hi = np.abs(parity.f64(o) - ref_o)
     e_sum = np.abs(parity.f64(o) + parity.f64(dev["o_lo"]) - ref_o)
-    assert e_sum.max() <= e_hi.max() and e_sum.mean() < 0.5 * e_hi.mean()
+    assert e_sum.max() <= e_hi.max() and e_sum.mean() < e_hi.mean()
     # without the residual the backward still runs (D from bf16 O alone)
     dq, dk, dv = ops.attention_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["dout"],
                                    inp.workload.scale, True)
