@@ -296,9 +296,10 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
   }
   const long gtid = blockIdx.x * (long)blockDim.x + threadIdx.x;
   const long gstride = (long)gridDim.x * blockDim.x;
-  // the fp16 copies
+  // the fp16 copies of Q, K, V (dO's is written by the D pass below, which
+  // reads every dO row anyway)
 #pragma unroll 1
-  for (int t = 0; t < 4; ++t) {
+  for (int t = 0; t < 3; ++t) {
     const __nv_bfloat16* src = t == 0 ? p.q : t == 1 ? p.k : t == 2 ? p.v : p.dout;
     __half* dst = t == 0 ? p.q16 : t == 1 ? p.k16 : t == 2 ? p.v16 : p.do16;
     const float sx = t == 0 ? s_sc.sq : t == 1 ? s_sc.sk : t == 2 ? s_sc.sv : s_sc.sdo;
@@ -340,6 +341,7 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
       const uint32_t av[4] = {a.x, a.y, a.z, a.w};
       const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
       const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
+      uint32_t h16[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         // O = bf16(O) + residual: exact in fp32 (about 16 significant bits)
@@ -348,7 +350,10 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
         const float2 y = unpack_bf16(bv[e]);
         s = fmaf(x.x + xr.x, y.x, s);
         s = fmaf(x.y + xr.y, y.y, s);
+        h16[e] = pack_f16(y.x * s_sc.sdo, y.y * s_sc.sdo);
       }
+      *reinterpret_cast<uint4*>(p.do16 + row * D + li * 8) =
+          make_uint4(h16[0], h16[1], h16[2], h16[3]);
     }
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
