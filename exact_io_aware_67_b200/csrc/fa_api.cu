@@ -3,6 +3,7 @@
 // include/fa.h.  The library allocates no device memory (the one exception
 // is the fixed scratch array behind fa_bwd_noalloc, a file-scope device
 // variable) and never synchronises the caller's stream.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -142,9 +143,26 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   const int smem = fa::FwdLayout<D>::ALLOC;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // dispatch chunks (see the kernel): one chunk of every (sequence, kv head)
+  // pair unless K and V together are at least twice the L2; then the fewest
+  // pairs whose blocks make at least two waves (one block per SM)
+  fa::FwdParams pc = p;
+  {
+    int dev = 0, sms = 0, l2 = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
+    if (e != cudaSuccess) return e;
+    const long npairs = (long)p.B * p.Hkv;
+    const long per_pair = (long)p.group * p.num_qblocks;
+    const double kv_bytes = 2.0 * (double)p.total * p.Hkv * D * 2.0;
+    const long want = (2L * sms + per_pair - 1) / per_pair;
+    pc.order_chunk = (kv_bytes >= 2.0 * l2) ? (int)std::max(1L, std::min(npairs, want))
+                                            : (int)npairs;
+  }
   const unsigned grid = (unsigned)p.num_qblocks * p.Hq * p.B;
   if (t_prof_begin != nullptr) cudaEventRecord(t_prof_begin, stream);
-  kern<<<grid, fa::FWD_THREADS, smem, stream>>>(mq, mk, mv, p);
+  kern<<<grid, fa::FWD_THREADS, smem, stream>>>(mq, mk, mv, pc);
   e = cudaGetLastError();
   if (e == cudaSuccess && t_prof_end != nullptr) e = cudaEventRecord(t_prof_end, stream);
   return e;

@@ -49,6 +49,7 @@ struct FwdParams {
   int B, Hq, Hkv, N, group;
   int total;               // token rows of a varlen batch
   int num_qblocks;         // ceil(N / 256)
+  int order_chunk;         // (sequence, kv head) pairs per dispatch chunk
   float scale_log2;        // scale * log2(e)
   unsigned long long wait_limit_ns;
   // block-sparse mode only: tile (qt, kt) of sequence b and kv head hk is

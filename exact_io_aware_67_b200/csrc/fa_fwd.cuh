@@ -110,10 +110,24 @@ __global__ void __launch_bounds__(FWD_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   // ---------------------------------------------------------------- work item
-  const int bh = p.B * p.Hq;
-  const int qb = p.num_qblocks - 1 - (int)(blockIdx.x / bh);   // heaviest blocks first
-  const int h = (int)(blockIdx.x % bh) % p.Hq;
-  const int b = (int)(blockIdx.x % bh) / p.Hq;
+  // The (sequence, kv head) pairs are cut into chunks of order_chunk pairs
+  // (with their query heads); within a chunk the Q block index is slowest,
+  // heaviest blocks first.  One chunk of every pair unless the K and V of all
+  // pairs are at least twice the L2: then a chunk holds at least two waves of
+  // blocks and the blocks in flight share the chunk's K/V tiles in L2 (at
+  // B=1, H=16, N=65536, d=128 the K/V set is 512 MiB).
+  const unsigned g = (unsigned)p.group;
+  const unsigned npairs = (unsigned)(p.B * p.Hkv);
+  const unsigned chunk = (unsigned)p.order_chunk;
+  const unsigned per_pair = g * (unsigned)p.num_qblocks;
+  const unsigned cidx = blockIdx.x / (chunk * per_pair);
+  const unsigned rr = blockIdx.x - cidx * chunk * per_pair;
+  const unsigned pairs = min(chunk, npairs - cidx * chunk);
+  const int qb = p.num_qblocks - 1 - (int)(rr / (pairs * g));   // heaviest blocks first
+  const unsigned rem = rr % (pairs * g);
+  const unsigned pair = cidx * chunk + rem / g;
+  const int b = (int)(pair / (unsigned)p.Hkv);
+  const int h = (int)((pair % (unsigned)p.Hkv) * g + rem % g);
   int seq_start = 0, len = p.N, bcoord = b;
   if (p.cu_seqlens != nullptr) {
     seq_range(p.cu_seqlens, b, p.total, &seq_start, &len);
