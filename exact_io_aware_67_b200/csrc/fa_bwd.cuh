@@ -475,9 +475,6 @@ struct BwdLayout {
 // warps 0-7: elementwise (two warpgroups, 64 query columns each)
 // warps 8-11: dQ drain;  warp 12: TMA producer;  warp 13: MMA issuer;
 // warps 14-15: idle (they only give their registers to the drain warps)
-#ifndef FA_BWD_POLY_OF_8
-#define FA_BWD_POLY_OF_8 0
-#endif
 constexpr int BWD_THREADS = 512;
 constexpr int BWD_REGS_DRAIN = 176;   // warpgroup 2 after setmaxnreg.inc
 constexpr int BWD_REGS_CTRL = 80;     // warpgroup 3 after setmaxnreg.dec
@@ -912,19 +909,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const float2 x23 = ffma2(make_float2(__uint_as_float(sv[4 * c4 + 2]),
                                                __uint_as_float(sv[4 * c4 + 3])),
                                    c22, make_float2(l4.z, l4.w));
-          if ((c4 & 7) >= 8 - FA_BWD_POLY_OF_8) {
-            // part of the exponentials on the FMA pipe (ex2_poly2)
-            const float2 p01 = ex2_poly2(x01), p23 = ex2_poly2(x23);
-            P[4 * c4 + 0] = p01.x;
-            P[4 * c4 + 1] = p01.y;
-            P[4 * c4 + 2] = p23.x;
-            P[4 * c4 + 3] = p23.y;
-          } else {
-            P[4 * c4 + 0] = ex2(x01.x);
-            P[4 * c4 + 1] = ex2(x01.y);
-            P[4 * c4 + 2] = ex2(x23.x);
-            P[4 * c4 + 3] = ex2(x23.y);
-          }
+          P[4 * c4 + 0] = ex2(x01.x);
+          P[4 * c4 + 1] = ex2(x01.y);
+          P[4 * c4 + 2] = ex2(x23.x);
+          P[4 * c4 + 3] = ex2(x23.y);
         }
         // masks (warp-uniform test first): causal diagonal tile -- key row
         // kv_row is masked for query q < kv_row -- and key rows past the end
