@@ -38,6 +38,7 @@ class Workload:
     scale: float
     varlen: Optional[tuple] = None   # (lo, hi) inclusive length range
     x8_row: bool = False             # scale one query row per head by 8
+    x8_key_row: bool = False         # scale one key row per kv head by 8
     seed: int = 0
     note: str = ""
 
@@ -48,6 +49,8 @@ class Workload:
             out["varlen_lengths"] = list(self.varlen)
         if self.x8_row:
             out["x8_query_row_per_head"] = True
+        if self.x8_key_row:
+            out["x8_key_row_per_kv_head"] = True
         return out
 
 
@@ -81,6 +84,7 @@ class Inputs:
     workload: Workload
     x8_rows: Optional[torch.Tensor] = None   # [B, Hq] row index scaled by 8
     lengths: Optional[list] = field(default=None)
+    x8_key_rows: Optional[torch.Tensor] = None   # [B, Hkv] key row index scaled by 8
 
     @property
     def total(self):
@@ -115,17 +119,26 @@ def generate(w: Workload, with_dout: bool = True) -> Inputs:
         for b in range(w.B):
             for h in range(w.Hq):
                 q[b, int(x8[b, h]), h, :] *= 8.0
+    x8k = None
+    if w.x8_key_row:
+        if w.varlen:
+            raise ValueError("x8 rows are defined for dense workloads only")
+        x8k = torch.randint(0, w.N, (w.B, w.Hkv), generator=g, dtype=torch.int64)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                k[b, int(x8k[b, h]), h, :] *= 8.0
     bf = torch.bfloat16
     return Inputs(q=q.to(bf), k=k.to(bf), v=v.to(bf),
                   dout=None if dout is None else dout.to(bf),
-                  cu_seqlens=cu, workload=w, x8_rows=x8, lengths=lengths)
+                  cu_seqlens=cu, workload=w, x8_rows=x8, lengths=lengths, x8_key_rows=x8k)
 
 
-def custom(name, B, Hq, Hkv, N, d, causal, scale=None, varlen=None, x8_row=False, seed=0):
+def custom(name, B, Hq, Hkv, N, d, causal, scale=None, varlen=None, x8_row=False, seed=0,
+           x8_key_row=False):
     """An ad-hoc workload (tests use this for edge shapes)."""
     return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, causal=causal,
                     scale=(1.0 / math.sqrt(d)) if scale is None else scale,
-                    varlen=varlen, x8_row=x8_row, seed=seed)
+                    varlen=varlen, x8_row=x8_row, x8_key_row=x8_key_row, seed=seed)
 
 
 def from_lengths(name, lengths, Hq, Hkv, d, causal, seed=0):

@@ -150,3 +150,29 @@ def test_calls_from_another_host_thread():
     assert "e" not in box, box.get("e")
     g = parity.oracle_bwd(inp)
     parity.assert_close("dQ", parity.f64(box["g"][0]), g["dq"])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_x8_key_row_relative(d, causal):
+    """One key row per (batch, kv head) scaled by 8 draws weight from about
+    half the query rows, so dV and dK on that row reach magnitudes where
+    bf16 rounding alone exceeds the absolute bar; such a case is judged by
+    relative error: every output within 1e-2 of its largest oracle
+    magnitude, and the mean error within 1e-3 of it."""
+    inp = workloads.generate(workloads.custom("x8k", 1, 4, 2, 1024, d, causal, x8_key_row=True))
+    ops.fa_clear_device_error()
+    o, lse, dq, dk, dv = _run(inp)
+    g = parity.oracle_bwd(inp)
+    # the scaled rows carry the largest dV entries, as the case intends
+    kr = inp.x8_key_rows.numpy()
+    dv_ref = np.abs(g["dv"])
+    assert all(dv_ref[0, kr[0, h], h].max() >= 0.5 * dv_ref[0, :, h].max() for h in range(2))
+    for nm, got, ref in (("O", o, g["o"]), ("dQ", dq, g["dq"]), ("dK", dk, g["dk"]),
+                         ("dV", dv, g["dv"])):
+        err = np.abs(parity.f64(got) - ref)
+        scale = np.abs(ref).max()
+        assert err.max() <= 1e-2 * scale, "%s: max error %.3e, max |ref| %.3e" % (
+            nm, err.max(), scale)
+        assert err.mean() <= 1e-3 * scale, "%s: mean error %.3e" % (nm, err.mean())
+    np.testing.assert_allclose(parity.f64(lse), g["lse"], atol=parity.TOL_LSE, rtol=0)

@@ -68,6 +68,18 @@ def test_generator_is_deterministic_and_ordered():
     for x, y in ((a.q, b.q), (a.k, b.k), (a.v, b.v), (a.dout, b.dout)):
         assert (x.float() == y.float()).all()
     assert a.x8_rows.shape == (1, 2)
+    # the key-row variant draws the same Q, K, V, dO and scales exactly one K
+    # row per (batch, kv head) by 8, leaving the query rows alone
+    wk = workloads.custom("tk", 2, 4, 2, 16, 8, True, x8_key_row=True)
+    ck = workloads.generate(wk)
+    c0 = workloads.generate(workloads.custom("tk", 2, 4, 2, 16, 8, True))
+    assert (ck.q.float() == c0.q.float()).all() and (ck.v.float() == c0.v.float()).all()
+    ratio_rows = (ck.k.float() != c0.k.float()).any(dim=-1)      # [B, N, Hkv]
+    for bb in range(2):
+        for h in range(2):
+            r = int(ck.x8_key_rows[bb, h])
+            assert ratio_rows[bb, :, h].nonzero().flatten().tolist() in ([r], [])
+            assert (ck.k[bb, r, h].float() == 8 * c0.k[bb, r, h].float()).all()
     wv = workloads.WORKLOADS["bert_large_varlen_32x128to512_h16_d64"]
     iv = workloads.generate(wv)
     assert len(iv.lengths) == 32 and all(128 <= L <= 512 for L in iv.lengths)
