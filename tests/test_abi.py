@@ -3,6 +3,8 @@ rejects bad arguments on the host before touching the device (CPU only)."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -141,3 +143,33 @@ def test_blockmask_rejects_bad_arguments(lib):
     g = ops.fa_bwd_blockmask(*([p] * 5), None, *([p] * 4), p, need, 1, 2, 2, 256, 64, 0.125, 1,
                              None, 0, 0, None)
     assert g == 1
+
+
+def _run_python(code, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=300)
+
+
+def test_missing_library_fails_loudly():
+    # no fallback: without the CUDA library the binding raises
+    r = _run_python("from exact_io_aware_67_b200 import ops\n"
+                    "try:\n"
+                    "    ops.load()\n"
+                    "except RuntimeError as e:\n"
+                    "    print('raised', e)\n",
+                    {"FA_LIBRARY_PATH": "/nonexistent/libfa.so"})
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.startswith("raised"), r.stdout
+
+
+def test_product_path_does_not_import_the_oracle():
+    # the package and its binding never load the oracle (test infrastructure)
+    r = _run_python("import sys\n"
+                    "import exact_io_aware_67_b200\n"
+                    "from exact_io_aware_67_b200 import ops, workloads, flops\n"
+                    "ops.load()\n"
+                    "print(sorted(m for m in sys.modules if m == 'oracle' or m.startswith('oracle.')))\n")
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "[]", r.stdout
