@@ -221,7 +221,7 @@ def rows_for_seconds(w, seconds, nthreads):
     probe = max(64, nthreads * 16)
     dt, _, _ = cpu_rows_sample(w, probe, nthreads, seed=12345)
     rate = probe / max(dt, 1e-6)
-    return max(probe, int(rate * seconds))
+    return max(nthreads, int(rate * seconds))
 
 
 def cpu_per_core(w):
@@ -236,9 +236,11 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     cores = len(os.sched_getaffinity(0))
-    # each step is a bounded sample (about 3 s of oracle time), so that the
-    # whole --steps/--warmup run stays within a few minutes
-    nrows = rows_for_seconds(w, 3.0, cores)
+    # each step is a bounded sample (about 3 s of oracle time, less when
+    # many steps are asked for), so that the whole --steps/--warmup run stays
+    # within about three minutes
+    per_step_s = min(3.0, max(0.1, 150.0 / max(1, args.steps + args.warmup)))
+    nrows = rows_for_seconds(w, per_step_s, cores)
     for it in range(args.warmup):
         cpu_rows_sample(w, nrows, cores, seed=1000 + it)
     times, flops, desc = [], [], ""

@@ -158,7 +158,7 @@ def fa_bwd_workspace_size(B, Hq, N, d, total_tokens):
 
 
 def fa_validate_cu_seqlens(cu_seqlens, B, N, total_tokens, stream):
-    """Enqueue the device-side check of a cu_seqlens array; its verdict is
+    """Enqueue the device-side check of a cu_seqlens array; its result is
     read with fa_device_error() after a synchronise (see include/fa.h)."""
     return load().fa_validate_cu_seqlens(cu_seqlens, B, N, total_tokens, stream)
 
