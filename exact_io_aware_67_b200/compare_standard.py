@@ -11,6 +11,14 @@ both on the same inputs and prints one JSON line per (N, d):
         [--dims 64,128] [--heads 16] [--causal] [--steps 10] [--warmup 3]
         [--only both|standard|flash]
 
+Besides the times, each side's device memory beyond its inputs is measured
+(the peak the allocator saw during one call): S and P make it grow as N^2
+for standard attention, against O and LSE, linear in N, for the tiled
+forward (paper review 结果; "注意力机制基础" 2.2.2's memory column).  When
+S and P (2 heads N^2 bf16) exceed the free device memory less a 4 GiB
+margin, the standard side is skipped and reports the bytes it would need,
+so that no allocation is ever made to fail; the tiled side still runs.
+
 Times are CUDA events on the launching stream, after warm-up.  Between timed
 iterations the L2 cache is flushed by writing a buffer larger than it, so
 that small problems do not run from L2.  The standard pipeline is
@@ -55,12 +63,34 @@ def _time(fn, steps, warmup, flush):
     return ts[len(ts) // 2]
 
 
+def _extra_bytes(fn):
+    """Peak device memory one call of fn allocates beyond what was live."""
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    r = fn()
+    torch.cuda.synchronize()
+    peak = torch.cuda.max_memory_allocated() - base
+    del r
+    return peak
+
+
 def run(N, d, heads, causal, steps, warmup, only, flush):
     g = torch.Generator(device="cuda").manual_seed(N * 1000 + d)
     q, k, v = (torch.randn((1, heads, N, d), generator=g, device="cuda").to(torch.bfloat16)
                for _ in range(3))
     scale = d ** -0.5
     out = {"N": N, "d": d, "heads": heads, "batch": 1, "causal": bool(causal)}
+    if only in ("both", "standard"):
+        need = 2 * heads * N * N * 2          # S and P, bf16
+        free, _ = torch.cuda.mem_get_info()
+        if need > free - (4 << 30):
+            out["standard_skipped_bytes_needed"] = need
+            out["device_free_bytes"] = free
+            only = "flash"
+        else:
+            out["standard_extra_bytes"] = _extra_bytes(
+                lambda: ops.standard_attention_fwd(q, k, v, scale, causal))
     if only in ("both", "standard"):
         ms = _time(lambda: ops.standard_attention_fwd(q, k, v, scale, causal), steps, warmup,
                    flush)
@@ -90,6 +120,8 @@ def run(N, d, heads, causal, steps, warmup, only, flush):
         del s, p, lse
     if only in ("both", "flash"):
         qt, kt, vt = (t.transpose(1, 2).contiguous() for t in (q, k, v))   # [1, N, H, d]
+        out["flash_extra_bytes"] = _extra_bytes(lambda: ops.attention_fwd(qt, kt, vt, scale,
+                                                                          causal))
         fms = _time(lambda: ops.attention_fwd(qt, kt, vt, scale, causal), steps, warmup, flush)
         out["flash_fwd_ms"] = fms
         out["flash_model_bytes"] = heads * 2 * (4 * N * d) + heads * 4 * N
