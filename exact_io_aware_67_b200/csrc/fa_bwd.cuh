@@ -208,15 +208,25 @@ __global__ void __launch_bounds__(256) bwd_absmax_kernel(const BwdParams p, long
     const long n8 = tokens * heads * (D / 8);
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     float m = 0.f;
-    for (long i = gtid; i < n8; i += gstride) {
-      const uint4 a = s4[i];
+    auto take = [&](const uint4 a) {
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 x = unpack_bf16(w[e]);
         m = fmaxf(m, fmaxf(fabsf(x.x), fabsf(x.y)));
       }
+    };
+    // four independent 16-byte loads in flight per thread: one at a time
+    // left HBM about half idle (2.9 TB/s on 50 MB)
+    long i = gtid;
+    for (; i + 3 * gstride < n8; i += 4 * gstride) {
+      uint4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = s4[i + u * gstride];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) take(a[u]);
     }
+    for (; i < n8; i += gstride) take(s4[i]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     mx[t] = m;
@@ -266,7 +276,7 @@ __device__ __forceinline__ BwdScales bwd_make_scales(const BwdParams& p, const f
 // scales (block 0 also stores them for the later kernels), then writes its
 // share of the four fp16 copies, D and the zeroed accumulator.
 template <int D>
-__global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long tokens) {
+__global__ void __launch_bounds__(256, 6) bwd_pre_kernel(const BwdParams p, long tokens) {
   __shared__ float red[8][4];
   __shared__ BwdScales s_sc;
   {
@@ -307,13 +317,20 @@ __global__ void __launch_bounds__(256, 8) bwd_pre_kernel(const BwdParams p, long
     const long n8 = tokens * heads * (D / 8);
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
-    for (long i = gtid; i < n8; i += gstride) {
-      const uint4 a = s4[i];
+    auto conv = [&](const uint4 a) {
       const float2 x0 = unpack_bf16(a.x), x1 = unpack_bf16(a.y);
       const float2 x2 = unpack_bf16(a.z), x3 = unpack_bf16(a.w);
-      d4[i] = make_uint4(pack_f16(x0.x * sx, x0.y * sx), pack_f16(x1.x * sx, x1.y * sx),
-                         pack_f16(x2.x * sx, x2.y * sx), pack_f16(x3.x * sx, x3.y * sx));
+      return make_uint4(pack_f16(x0.x * sx, x0.y * sx), pack_f16(x1.x * sx, x1.y * sx),
+                        pack_f16(x2.x * sx, x2.y * sx), pack_f16(x3.x * sx, x3.y * sx));
+    };
+    // two independent loads in flight per thread
+    long i = gtid;
+    for (; i + gstride < n8; i += 2 * gstride) {
+      const uint4 a0 = s4[i], a1 = s4[i + gstride];
+      d4[i] = conv(a0);
+      d4[i + gstride] = conv(a1);
     }
+    if (i < n8) d4[i] = conv(s4[i]);
   }
   // zero the accumulator
   {
@@ -1029,7 +1046,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUt
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: absmax kernel launch\n");
     return e;
   }
-  bwd_pre_kernel<D><<<sms * 8, 256, 0, stream>>>(pp, tokens);
+  bwd_pre_kernel<D><<<sms * 6, 256, 0, stream>>>(pp, tokens);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     if (std::getenv("FA_DEBUG")) std::fprintf(stderr, "libfa: pre kernel launch\n");
